@@ -1,0 +1,308 @@
+"""Pins for the CPU oracle: what the pages and the mathematics fix, checked
+against something other than the oracle itself (hand-worked fixtures, closed
+forms, invariants, brute force, library routines, error bounds).
+
+Method: Keras guide "INT4 quantization in Keras", section "How it works",
+steps 1-6; the minimal model of section "Quantize a minimal functional model".
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.conftest import read_golden
+from w4a8_quantized_gemm_channel_b200 import synth
+
+
+def _ints(vals):
+    return [int(v) for v in vals]
+
+
+# ---------------------------------------------------------------- packing ---
+
+def test_pack_matches_hand_worked_bytes():
+    """The nibble order and two's-complement encoding, worked by hand for
+    every code value in both nibble positions, plus an odd K."""
+    rows = read_golden("pack_codes.txt")
+    assert len(rows) % 2 == 0 and rows
+    for (k1, codes), (k2, hexbytes) in zip(rows[::2], rows[1::2]):
+        assert k1 == "codes" and k2 == "bytes"
+        q = np.array([_ints(codes)], np.int8)
+        wp = oracle.w4_pack(q)
+        want = bytes(int(h, 16) for h in hexbytes)
+        assert wp.shape[1] == oracle.packed_ld(q.shape[1])
+        assert bytes(wp[0, :len(want)]) == want
+        assert not wp[0, len(want):].any(), "pad bytes must be zero"
+        # and unpacking gives the codes back
+        assert np.array_equal(oracle.w4_unpack(wp, q.shape[1]), q)
+
+
+def test_pack_unpack_round_trip_exhaustive():
+    """unpack(pack(q)) == q for every pair of codes in [-8, 7], and
+    pack(unpack(b)) == b for every byte value."""
+    pairs = np.array(list(itertools.product(range(-8, 8), repeat=2)), np.int8)  # 256 x 2
+    wp = oracle.w4_pack(pairs)
+    assert np.array_equal(oracle.w4_unpack(wp, 2), pairs)
+    # every byte value occurs exactly once among the packed pairs
+    assert sorted(wp[:, 0].tolist()) == list(range(256))
+    allbytes = np.zeros((256, 16), np.uint8)
+    allbytes[:, 0] = np.arange(256)
+    q = oracle.w4_unpack(allbytes, 2)
+    assert q.min() == -8 and q.max() == 7
+    assert np.array_equal(oracle.w4_pack(q)[:, 0], np.arange(256))
+
+
+def test_packed_size_is_params_times_bits_over_8():
+    """Size = parameters x 4 bits / 8 (the concept page's storage formula),
+    before the row padding to 16 bytes."""
+    for k in (1, 2, 3, 31, 32, 33, 4096, 6912):
+        assert oracle.packed_ld(k) >= math.ceil(k * 4 / 8)
+        assert oracle.packed_ld(k) - math.ceil(k * 4 / 8) < 16
+        assert oracle.packed_ld(k) % 16 == 0
+
+
+# --------------------------------------------------------------- rounding ---
+
+def test_weight_ties_round_half_even():
+    g = dict(read_golden("round_half_even.txt"))
+    w = np.array([float(v) for v in g["weight_column"]], np.float32)[:, None]
+    q, sw = oracle.w4_quantize(w)
+    assert sw[0] == np.float32(1.0)
+    assert q[0].tolist() == _ints(g["weight_codes"])
+
+
+def test_activation_ties_round_half_even():
+    g = dict(read_golden("round_half_even.txt"))
+    x = np.array([[float(v) for v in g["act_row"]]], np.float32)
+    xq, sx = oracle.a8_quantize_rows(x)
+    assert sx[0] == np.float32(1.0)
+    assert xq[0].tolist() == _ints(g["act_codes"])
+
+
+# ------------------------------------------------------ weight quantization ---
+
+def _random_w(k=384, n=96, seed=11):
+    return synth.linear_weights(k, n, 0.02, seed)
+
+
+def test_weight_codes_in_range_and_extremes_hit_7():
+    """Codes stay in [-8, 7]; with abs-max scaling to 7 they never reach -8,
+    and the element attaining a column's abs-max maps to exactly +-7."""
+    w = _random_w()
+    q, sw = oracle.w4_quantize(w)
+    assert q.min() >= -7 and q.max() <= 7
+    for n in range(w.shape[1]):
+        kmax = int(np.argmax(np.abs(w[:, n])))
+        assert q[n, kmax] == (7 if w[kmax, n] > 0 else -7)
+    # the scale is 7 / abs-max (float32 division)
+    amax = np.abs(w).max(axis=0)
+    assert np.array_equal(sw, (np.float32(7.0) / amax).astype(np.float32))
+
+
+def test_weight_scale_invariance_by_powers_of_two():
+    """Scaling a column by 2^j leaves its codes unchanged and divides its
+    scale by exactly 2^j (both products are exact in binary floating point)."""
+    w = _random_w(k=200, n=8, seed=12)
+    q0, sw0 = oracle.w4_quantize(w)
+    for j in (-3, 1, 5):
+        wj = (w * np.float32(2.0 ** j)).astype(np.float32)
+        qj, swj = oracle.w4_quantize(wj)
+        assert np.array_equal(qj, q0)
+        assert np.array_equal(swj * np.float32(2.0 ** j), sw0)
+
+
+def test_weight_sign_symmetry():
+    """Round-half-even is odd-symmetric, so Q(-W) = -Q(W) with the same scale."""
+    w = _random_w(k=256, n=16, seed=13)
+    q0, sw0 = oracle.w4_quantize(w)
+    q1, sw1 = oracle.w4_quantize(-w)
+    assert np.array_equal(sw0, sw1)
+    assert np.array_equal(q1, -q0)
+
+
+def test_zero_column_and_zero_row():
+    w = _random_w(k=64, n=4, seed=14)
+    w[:, 2] = 0.0
+    q, sw = oracle.w4_quantize(w)
+    assert sw[2] == np.float32(1.0) and not q[2].any()
+    x = synth.normal((3, 64), 1.0, synth.rng_for(14, 9))
+    x[1] = 0.0
+    xq, sx = oracle.a8_quantize_rows(x)
+    assert sx[1] == np.float32(1.0) and not xq[1].any()
+
+
+def test_weight_error_bound():
+    """|w - q/sw| <= 0.5/sw for every element: no value is clipped (the
+    abs-max maps to 7 < 8), so rounding is the only error."""
+    w = _random_w(k=512, n=64, seed=15).astype(np.float64)
+    q, sw = oracle.w4_quantize(w.astype(np.float32))
+    sw64 = sw.astype(np.float64)
+    err = np.abs(w.T - q.astype(np.float64) / sw64[:, None])
+    bound = 0.5 / sw64[:, None] * (1 + 1e-6)
+    assert (err <= bound).all()
+
+
+# -------------------------------------------------- activation quantization ---
+
+def test_activation_codes_range_extremes_and_error_bound():
+    x, _ = synth.linear_activations(16, 1000, seed=16, outlier_count=5, outlier_factor=20.0)
+    xq, sx = oracle.a8_quantize_rows(x)
+    assert xq.min() >= -127 and xq.max() <= 127
+    for m in range(x.shape[0]):
+        k = int(np.argmax(np.abs(x[m])))
+        assert xq[m, k] == (127 if x[m, k] > 0 else -127)
+    assert np.array_equal(sx, (np.float32(127.0) / np.abs(x).max(axis=1)).astype(np.float32))
+    err = np.abs(x.astype(np.float64) - xq.astype(np.float64) / sx.astype(np.float64)[:, None])
+    assert (err <= 0.5 / sx.astype(np.float64)[:, None] * (1 + 1e-6)).all()
+
+
+def test_activation_pad_bytes_are_zero():
+    x = synth.normal((5, 37), 1.0, synth.rng_for(17, 1))
+    xq, _ = oracle.a8_quantize_rows(x, ldq=48)
+    assert not xq[:, 37:].any()
+
+
+# ---------------------------------------------------------------- the GEMM ---
+
+def test_gemm_brute_force_exhaustive_tiny():
+    """Every weight code vector in [-8, 7]^K for K <= 3 against fixed
+    activation rows (extremes included), checked with a pure-Python loop."""
+    for k in (1, 2, 3):
+        q = np.array(list(itertools.product(range(-8, 8), repeat=k)), np.int8)  # N x K
+        xq = np.array([[127] * k, [-127] * k, list(range(1, k + 1)),
+                       [(-1) ** i * (30 + 11 * i) for i in range(k)]], np.int8)
+        acc = oracle.gemm_s32(xq, k, oracle.w4_pack(q))
+        for m in range(xq.shape[0]):
+            for n in range(q.shape[0]):
+                s = 0
+                for kk in range(k):
+                    s += int(xq[m, kk]) * int(q[n, kk])
+                assert acc[m, n] == s
+
+
+def test_gemm_brute_force_small_random():
+    rng = synth.rng_for(18, 0)
+    for (m, k, n) in ((1, 1, 1), (3, 7, 5), (4, 8, 4), (2, 33, 3)):
+        q = rng.integers(-8, 8, size=(n, k)).astype(np.int8)
+        xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+        acc = oracle.gemm_s32(xq, k, oracle.w4_pack(q))
+        want = [[sum(int(xq[i, t]) * int(q[j, t]) for t in range(k)) for j in range(n)]
+                for i in range(m)]
+        assert acc.tolist() == want
+
+
+def test_gemm_matches_float64_matmul_medium():
+    """Integer products summed in float64 are exact while |acc| < 2^53."""
+    rng = synth.rng_for(19, 0)
+    m, k, n = 24, 777, 40
+    q = rng.integers(-8, 8, size=(n, k)).astype(np.int8)
+    xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+    acc = oracle.gemm_s32(xq, k, oracle.w4_pack(q))
+    ref = xq.astype(np.float64) @ q.astype(np.float64).T
+    assert np.array_equal(acc.astype(np.float64), ref)
+
+
+def test_gemm_int32_overflow_is_reported():
+    k = 2_200_000  # 127 * 8 * k > 2^31
+    xq = np.full((1, k), -127, np.int8)
+    q = np.full((1, k), -8, np.int8)
+    with pytest.raises(oracle.OracleError):
+        oracle.gemm_s32(xq, k, oracle.w4_pack(q))
+
+
+# --------------------------------------------------------- dequantization ---
+
+def test_dequant_direction_exact_powers_of_two():
+    """With abs-maxes 3.5 and 63.5 both scales are exactly 2, every value is a
+    half-integer and exactly representable, so y must equal X @ W exactly:
+    y = acc / (sx * sw) = acc / 4. Dividing by sx/sw or multiplying by
+    sx*sw instead would miss by a factor of 4 or 16."""
+    rng = synth.rng_for(20, 0)
+    m, k, n = 6, 50, 9
+    wq = rng.integers(-7, 8, size=(k, n)).astype(np.float32)
+    wq[0, :] = 7
+    xq = rng.integers(-127, 128, size=(m, k)).astype(np.float32)
+    xq[:, 0] = 127
+    w = wq / 2   # abs-max 3.5 -> sw = 2
+    x = xq / 2   # abs-max 63.5 -> sx = 2
+    wp, sw = oracle.w4_quantize_pack(w)
+    assert (sw == 2.0).all()
+    y = oracle.linear(x, wp, sw, k)
+    exact = x.astype(np.float64) @ w.astype(np.float64)
+    assert np.array_equal(y.astype(np.float64), exact)
+
+
+def test_dequant_bias_and_relu():
+    acc = np.array([[-10, 0, 10, 3]], np.int32)
+    sx = np.array([2.0], np.float32)
+    sw = np.array([1.0, 1.0, 0.5, 4.0], np.float32)
+    b = np.array([4.0, -1.0, 0.5, 0.0], np.float32)
+    y = oracle.dequant(acc, sx, sw, b, relu=False)
+    assert y.tolist() == [[-1.0, -1.0, 10.5, 0.375]]
+    y = oracle.dequant(acc, sx, sw, b, relu=True)
+    assert y.tolist() == [[0.0, 0.0, 10.5, 0.375]]
+    assert not np.signbit(y).any()
+
+
+def test_end_to_end_error_bound():
+    """|y_q - y_exact| <= sum_k (|x_k| e_w + |w_k| e_x + e_w e_x) + float32
+    slack, with e_w = 0.5/sw and e_x = 0.5/sx and y_exact = X @ W in float64.
+    A swapped scale convention or a dropped factor breaks this bound."""
+    x, _ = synth.linear_activations(8, 640, seed=21, outlier_count=3, outlier_factor=20.0)
+    w = synth.linear_weights(640, 48, 0.02, seed=21)
+    wp, sw = oracle.w4_quantize_pack(w)
+    xq, sx = oracle.a8_quantize_rows(x)
+    y = oracle.linear(x, wp, sw, 640)
+    x64, w64 = x.astype(np.float64), w.astype(np.float64)
+    exact = x64 @ w64
+    ew = 0.5 / sw.astype(np.float64)            # [N]
+    ex = 0.5 / sx.astype(np.float64)            # [M]
+    bound = (np.abs(x64).sum(1)[:, None] * ew[None, :]
+             + ex[:, None] * np.abs(w64).sum(0)[None, :]
+             + 640 * ex[:, None] * ew[None, :])
+    slack = 1e-5 * (np.abs(x64) @ np.abs(w64)) + 1e-6
+    assert (np.abs(y - exact) <= bound + slack).all()
+    # and the error is not trivially zero: quantization happened
+    assert np.abs(y - exact).max() > 0
+
+
+def test_bf16_rounding_matches_torch():
+    """float32 -> bf16 round-to-nearest-even agrees with torch's conversion."""
+    rng = synth.rng_for(22, 0)
+    y = np.concatenate([rng.standard_normal(4096).astype(np.float32) * 100,
+                        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, -3.0e38, 1e-40],
+                                 np.float32)])
+    want = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.to_bf16_bits(y), want)
+
+
+# -------------------------------------------------------- minimal model ---
+
+def _fp_mlp(d: synth.MinimalMLP) -> np.ndarray:
+    x = d.x.astype(np.float64)
+    h = np.maximum(x @ d.w1.astype(np.float64) + d.b1, 0.0)
+    return h @ d.w2.astype(np.float64) + d.b2
+
+
+def test_minimal_model_mse_order_of_magnitude():
+    """The page's minimal model: quantized vs full-precision MSE is small and
+    of the order the page prints (its data are unseeded: order only)."""
+    page = float(dict(read_golden("minimal_mlp_mse.txt"))["page_mse"][0])
+    d = synth.minimal_mlp(seed=0)
+    yq = oracle.mlp(d.x, d.w1, d.b1, d.w2, d.b2)
+    mse = float(np.mean((_fp_mlp(d) - yq.astype(np.float64)) ** 2))
+    assert 0.0 < mse <= 1e-2
+    assert page / 100 <= mse <= page * 100, (mse, page)
+
+
+def test_minimal_model_is_deterministic():
+    """Re-running the quantized model gives bit-identical outputs (the page's
+    save/reload MSE is identical for the same reason: the quantized state is
+    just packed bytes and scales)."""
+    d = synth.minimal_mlp(seed=0)
+    a = oracle.mlp(d.x, d.w1, d.b1, d.w2, d.b2)
+    b = oracle.mlp(d.x, d.w1, d.b1, d.w2, d.b2)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
