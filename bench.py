@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A8 per-channel linear layer on B200.
+
+Default workload: the decode single linear, K = N = 4096, activation rows
+M in {1, 4, 16}. One step = one pass of the run-time hot path over one batch:
+for each M, dynamic INT8 quantization of X[M][4096] and the W4A8 product with
+dequantization (w4a8_linear: two kernels). The weights are quantized and
+packed once, offline, before timing (their quantize+pack pass is timed on its
+own and reported under "stages").
+
+Metric: HBM GB/s of algorithmic bytes (packed weights + weight scales +
+float32 X + float32 Y per linear) per second of device time. Weight buffers
+rotate through a pool of distinct copies several times larger than L2, so
+every launch streams its weights from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill]
+
+Multi-GPU (torchrun): every rank runs the same independent workload (weak
+scaling, no collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A8 linear: TOPS (prefill) and HBM GB/s (decode) vs B200 roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
+GRAPH_STEPS = 16
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- workloads ---
+
+class DecodeWorkload:
+    """K = N = 4096, M in {1, 4, 16}; weights N(0, 0.02), X N(0, 1) with 8
+    outlier channels x20."""
+    name = "decode"
+
+    def __init__(self, torch, native, synth, device, l2_bytes):
+        self.torch, self.nat = torch, native
+        self.K, self.N, self.MS = synth.DECODE_K, synth.DECODE_N, synth.DECODE_MS
+        w = synth.decode_case(1).w
+        self.w_host = w
+        wd = torch.from_numpy(w).to(device)
+        wp, sw = native.w4_quantize_pack(wd)
+        self.wd = wd
+        per_weight = wp.numel() + 4 * sw.numel()
+        # enough distinct copies (>= 3x L2) that each launch's weights were
+        # evicted from L2 since their last use
+        need = -(-3 * l2_bytes // per_weight) + len(self.MS)
+        self.pool = -(-need // len(self.MS)) * len(self.MS)
+        self.wp = [wp.clone() for _ in range(self.pool)]
+        self.sw = [sw.clone() for _ in range(self.pool)]
+        self.x_host = {m: synth.decode_case(m).x for m in self.MS}
+        self.x = {m: torch.from_numpy(self.x_host[m]).to(device) for m in self.MS}
+        self.y = {m: torch.empty((m, self.N), dtype=torch.float32, device=device) for m in self.MS}
+        self.ws = {m: torch.empty(native.workspace_size(m, self.K), dtype=torch.uint8, device=device)
+                   for m in self.MS}
+        self.slot = 0
+        self.pool_bytes = self.pool * per_weight
+
+    def bytes_per_step(self):
+        ldp = self.nat.packed_ld(self.K)
+        return sum(self.N * ldp + 4 * self.N + 4 * m * self.K + 4 * m * self.N for m in self.MS)
+
+    def ops_per_step(self):
+        return sum(2 * m * self.N * self.K for m in self.MS)
+
+    def launches_per_step(self):
+        return 2 * len(self.MS)
+
+    def step(self):
+        for m in self.MS:
+            s = self.slot
+            self.slot = (self.slot + 1) % self.pool
+            self.nat.w4a8_linear(self.x[m], self.wp[s], self.sw[s], y=self.y[m], workspace=self.ws[m])
+
+    def config(self):
+        return {"workload": f"decode single linear K={self.K} N={self.N} M in {list(self.MS)}",
+                "K": self.K, "N": self.N, "M": list(self.MS),
+                "l2": f"inputs larger than L2: {self.pool} distinct packed weight buffers "
+                      f"({self.pool_bytes / 1e6:.0f} MB) rotate across launches",
+                "weights": "N(0,0.02) quantized+packed once before timing",
+                "activations": "N(0,1), 8 input channels x20"}
+
+
+# ------------------------------------------------------------ timing core ---
+
+def build_graphs(torch, wl, nsteps):
+    """CUDA graphs of GRAPH_STEPS steps (and one for the remainder)."""
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):           # warm the library's per-device state outside capture
+            wl.step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    full, rem = divmod(nsteps, GRAPH_STEPS)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(GRAPH_STEPS):
+            wl.step()
+    gr = None
+    if rem:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for _ in range(rem):
+                wl.step()
+    return g, full, gr
+
+
+def time_steps(torch, wl, steps, warmup, dist=None):
+    g, full, gr = build_graphs(torch, wl, steps)
+    wg, wfull, wgr = build_graphs(torch, wl, warmup) if warmup else (None, 0, None)
+    for _ in range(wfull):
+        wg.replay()
+    if wgr is not None:
+        wgr.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(full):
+        g.replay()
+    if gr is not None:
+        gr.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = start.elapsed_time(stop)
+    return ms
+
+
+def time_kernel_only(torch, nat, wl):
+    """Average device time per decode-kernel launch (w4a8_linear_q, INT8
+    activations already quantized) in a back-to-back graph over the rotating
+    weight pool, per M; returns {m: (ms_per_launch, algorithmic_bytes)}."""
+    out = {}
+    ldp = nat.packed_ld(wl.K)
+    for m in wl.MS:
+        xq, sx = nat.a8_quantize_rows(wl.x[m])
+        reps = wl.pool
+
+        def run():
+            for i in range(reps):
+                nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], y=wl.y[m])
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run()
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_rep = 20
+        start.record()
+        for _ in range(n_rep):
+            g.replay()
+        stop.record()
+        torch.cuda.synchronize()
+        ms = start.elapsed_time(stop) / (n_rep * reps)
+        nbytes = wl.N * ldp + 4 * wl.N + m * xq.shape[1] + 4 * m + 4 * m * wl.N
+        out[m] = (ms, nbytes)
+    return out
+
+
+def time_quantize_pack(torch, nat, wl):
+    """The offline weight pass (steps 1-2) on the decode weight matrix."""
+    wp, sw = nat.w4_quantize_pack(wl.wd)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 20
+    start.record()
+    for _ in range(reps):
+        nat.w4_quantize_pack(wl.wd, wp=wp, sw=sw)
+    stop.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / reps
+    nbytes = wl.wd.numel() * 4 + wp.numel() + 4 * sw.numel()
+    return ms, nbytes
+
+
+def time_e2e(torch, nat, wl, steps):
+    """Same metric through the public call with host buffers: every step
+    copies X from pinned host memory and reads Y back."""
+    xh = {m: torch.from_numpy(wl.x_host[m]).pin_memory() for m in wl.MS}
+    yh = {m: torch.empty((m, wl.N), dtype=torch.float32).pin_memory() for m in wl.MS}
+    xd = {m: torch.empty_like(wl.x[m]) for m in wl.MS}
+
+    def one(slot):
+        for j, m in enumerate(wl.MS):
+            s = (slot * len(wl.MS) + j) % wl.pool
+            xd[m].copy_(xh[m], non_blocking=True)
+            nat.w4a8_linear(xd[m], wl.wp[s], wl.sw[s], y=wl.y[m], workspace=wl.ws[m])
+            yh[m].copy_(wl.y[m], non_blocking=True)
+    for i in range(5):
+        one(i)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        one(i)
+    stop.record()
+    torch.cuda.synchronize()
+    h2d = sum(xh[m].numel() * 4 for m in wl.MS)
+    d2h = sum(yh[m].numel() * 4 for m in wl.MS)
+    return start.elapsed_time(stop), h2d, d2h
+
+
+# ------------------------------------------------------- the CPU oracle ---
+
+def oracle_decode_rate(budget_s: float, min_steps: int = 1):
+    """The oracle as it stands, on a bounded sample of the decode workload:
+    all three M values against a sample of output channels (full K)."""
+    import oracle
+    from w4a8_quantized_gemm_channel_b200 import synth
+    k, n = synth.DECODE_K, synth.DECODE_N
+    w = synth.decode_case(1).w
+    xs = {m: synth.decode_case(m).x for m in synth.DECODE_MS}
+    wp, sw = oracle.w4_quantize_pack(w)
+    ldp = wp.shape[1]
+    cols = 64
+    done_bytes, t_used, chunks = 0, 0.0, 0
+    t0 = time.perf_counter()
+    while (time.perf_counter() - t0 < budget_s) or chunks < min_steps:
+        c0 = (chunks * cols) % n
+        wps, sws = wp[c0:c0 + cols], sw[c0:c0 + cols]
+        for m, x in xs.items():
+            oracle.linear(x, wps, sws, k)
+            done_bytes += cols * ldp + 4 * cols + 4 * m * k + 4 * m * cols
+        chunks += 1
+    t_used = time.perf_counter() - t0
+    return done_bytes / t_used / 1e9, t_used, chunks, cols
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    budget = min(120.0, max(10.0, 0.01 * (args.steps + args.warmup)))
+    gbs, t, chunks, cols = oracle_decode_rate(budget)
+    sample = (f"{chunks} samples of {cols} output channels x full K=4096 at M=1,4,16 "
+              f"({t:.1f} s single-threaded)")
+    line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "impl": "reference",
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "decode single linear K=4096 N=4096 M in [1, 4, 16]",
+                       "note": "CPU oracle (plain C, one thread) on a bounded sample"},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- main ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of CPU work for the oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(local)
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    # the CPU baseline runs before any GPU work on rank 0 only, at N = 1
+    cpu = None
+    if rank == 0 and world == 1:
+        gbs, t, chunks, cols = oracle_decode_rate(args.cpu_budget)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{chunks} samples of {cols} output channels x full K=4096 at M=1,4,16 "
+                         f"({t:.1f} s, single-threaded plain C)"}
+
+    from w4a8_quantized_gemm_channel_b200 import native, synth
+    props = torch.cuda.get_device_properties(device)
+    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_steps(torch, wl, args.steps, args.warmup, dist)
+    ck = clocks.stop()
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    bytes_step = wl.bytes_per_step()
+    value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9
+
+    kern = time_kernel_only(torch, native, wl)
+    k_ms = sum(v[0] for v in kern.values())
+    k_bytes = sum(v[1] for v in kern.values())
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    achieved = k_bytes / (k_ms * 1e-3) / 1e9
+    qp_ms, qp_bytes = time_quantize_pack(torch, native, wl)
+    e2e_steps = min(args.steps, 2000)
+    e2e_ms, h2d, d2h = time_e2e(torch, native, wl, e2e_steps)
+    e2e_val = world * e2e_steps * bytes_step / (e2e_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8xs4->s32",
+        "data": "synthetic", "config": wl.config(),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": None,
+                     "kernel": "k_linear_decode (w4a8_linear_q, back-to-back, rotating weights)",
+                     "per_m": {str(m): {"us": round(v[0] * 1e3, 3), "bytes": v[1],
+                                        "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
+                               for m, v in kern.items()}},
+        "stages": {"quantize_pack": {"ms": round(qp_ms, 4), "bytes": qp_bytes,
+                                     "gbs": round(qp_bytes / (qp_ms * 1e-3) / 1e9, 1),
+                                     "frac_hbm": round(qp_bytes / (qp_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                                     "shape": f"K={wl.K} N={wl.N} fp32 -> packed"}},
+        "tops": round(world * args.steps * wl.ops_per_step() / (ms * 1e-3) / 1e12, 4),
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * wl.launches_per_step(),
+        "clocks": ck,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,167 @@
+/*
+ * w4a8.h - C ABI of libw4a8.so, a B200 (sm_100a) implementation of the W4A8
+ * per-output-channel quantized linear layer.
+ *
+ * The operation is the one the Keras guide "INT4 quantization in Keras"
+ * describes in its section "How it works" (steps 1-6) and section "What Keras
+ * does in INT4 mode":
+ *   weights    - per-output-channel symmetric abs-max scale sw = 7 / max|W[:,n]|
+ *                (1 for an all-zero column), codes q = clamp(rne(w * sw), -8, 7),
+ *                packed two per byte along K, even k in the low nibble;
+ *   activations- per-row dynamic abs-max INT8: sx = 127 / max|X[m,:]| (1 for an
+ *                all-zero row), xq = clamp(rne(x * sx), -127, 127);
+ *   product    - INT4 codes unpacked to INT8, INT8 x INT8 accumulated in INT32;
+ *   output     - y = float(acc) / (sx * sw), then + bias[n], then ReLU if asked
+ *                (the Dense epilogue of the guide's minimal model, section
+ *                "Quantize a minimal functional model").
+ * "rne" is round to nearest, ties to even; every float operation is IEEE
+ * float32 round-to-nearest, so integer results are bit-exact and float32
+ * outputs match a float32 statement of the same steps.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates, never frees and never synchronizes the stream; work is
+ *    enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *    and the call returns once it is enqueued.
+ *  - Strides ("ld") count elements of the array's type: floats for W, X, Y
+ *    (f32), bf16 elements or int32 elements for Y in those formats, bytes for
+ *    Wp and Xq.
+ *  - Packed weights Wp and INT8 activations Xq must start on a 16-byte
+ *    boundary and have a stride that is a multiple of 16 bytes.
+ *  - Errors are returned as a w4a8_status; nothing is enqueued when an
+ *    argument check fails. A CUDA launch failure returns W4A8_ERR_CUDA.
+ *  - Kernels that detect an internal fault (an out-of-range index or a bounded
+ *    wait that ran out) record it in a per-device status word instead of
+ *    trapping; read it with w4a8_get_device_status after synchronizing.
+ */
+#ifndef W4A8_H
+#define W4A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W4A8_API __attribute__((visibility("default")))
+#else
+#define W4A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int w4a8_status;
+
+enum {
+    W4A8_OK = 0,
+    W4A8_ERR_INVALID_ARG = 1,  /* a null pointer, a bad size, stride or alignment */
+    W4A8_ERR_UNSUPPORTED = 2,  /* no sm_100 device, or a path forced on a shape it cannot run */
+    W4A8_ERR_WORKSPACE = 3,    /* workspace missing or smaller than w4a8_workspace_size() */
+    W4A8_ERR_CUDA = 4,         /* a CUDA runtime call failed (e.g. a launch) */
+    W4A8_ERR_TIMEOUT = 5,      /* (device status) a bounded wait inside a kernel ran out */
+    W4A8_ERR_BOUNDS = 6        /* (device status) a kernel caught an out-of-range index */
+};
+
+/* Flags of w4a8_linear / w4a8_linear_q. */
+#define W4A8_RELU          0x01u /* y = y > 0 ? y : +0 after the bias */
+#define W4A8_OUT_F32       0x00u /* Y is float32 [M][ldy] (default) */
+#define W4A8_OUT_BF16      0x02u /* Y is bfloat16 [M][ldy], rounded to nearest even */
+#define W4A8_OUT_S32       0x04u /* Y is the raw INT32 accumulator [M][ldy]; no bias, no ReLU */
+#define W4A8_OUT_MASK      0x06u
+/* Kernel selection. AUTO picks by shape; the others force one kernel (tests). */
+#define W4A8_PATH_AUTO     0x00u
+#define W4A8_PATH_GENERIC  0x10u /* CUDA-core kernel, any shape */
+#define W4A8_PATH_DECODE   0x20u /* weight-streaming kernel for few rows (M <= 16 per tile) */
+#define W4A8_PATH_TC       0x30u /* tcgen05 tensor-core GEMM (INT32 accumulators in TMEM) */
+#define W4A8_PATH_MASK     0x30u
+
+/* Largest K whose INT32 accumulator cannot overflow: 127 * 8 * K < 2^31. */
+#define W4A8_MAX_K 2097152
+
+/* Bytes per packed output-channel row: ceil(K/2) rounded up to a multiple of
+ * 16 (the stride every tensor-core tile load needs). Returns -1 if K < 1. */
+W4A8_API int w4a8_packed_ld(int K);
+
+/* Bytes per INT8 activation row used inside w4a8_linear: K rounded up to a
+ * multiple of 16. Returns -1 if K < 1. */
+W4A8_API int w4a8_act_ld(int K);
+
+/* Workspace bytes w4a8_linear needs for M rows of K inputs (the INT8
+ * activations and their scales). Returns 0 if M < 0 or K < 1. */
+W4A8_API size_t w4a8_workspace_size(int M, int K);
+
+/*
+ * w4_quantize_pack - steps 1-2 of "How it works": per-output-channel abs-max
+ * scale, half-even rounding to [-8, 7], two codes per byte.
+ *   W   [K][ldw] float32, row k = input feature k, column n = output channel n
+ *       (the Keras kernel layout), ldw >= N.
+ *   Wp  [N][ldp] bytes out, ldp >= ceil(K/2) and a multiple of 16: byte j of
+ *       row n = (q[n][2j] & 0xF) | (q[n][2j+1] & 0xF) << 4. Every byte past
+ *       the nibble of k = K-1 (the odd-K pad nibble included) is written 0.
+ *   sw  [N] float32 out: 7 / max_k |W[k][n]|, or 1 for an all-zero column.
+ * Requires 1 <= K <= W4A8_MAX_K, N >= 1. Inputs must be finite.
+ * Uses sw as scratch while it runs, so W and sw must not overlap.
+ */
+W4A8_API w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw,
+                             uint8_t *Wp, int ldp, float *sw, void *stream);
+
+/*
+ * a8_quantize_rows - step 3: dynamic per-row abs-max INT8 quantization.
+ *   X   [M][ldx] float32 (ldx >= K), finite.
+ *   Xq  [M][ldq] int8 out (ldq >= K, multiple of 16); bytes K..ldq-1 of each
+ *       row are written 0.
+ *   sx  [M] float32 out: 127 / max_k |X[m][k]|, or 1 for an all-zero row.
+ * M == 0 is a no-op returning W4A8_OK.
+ */
+W4A8_API w4a8_status a8_quantize_rows(const float *X, int M, int K, int ldx,
+                             int8_t *Xq, int ldq, float *sx, void *stream);
+
+/*
+ * w4a8_linear - steps 3-6 on float32 activations: quantize each row of X to
+ * INT8, multiply with the packed INT4 weights (unpacked to INT8 on chip),
+ * accumulate in INT32, dequantize, add the bias, apply ReLU.
+ *   X     [M][ldx] float32, ldx >= K.
+ *   Wp,sw as produced by w4_quantize_pack for this K and N (pad nibbles 0).
+ *   bias  [N] float32 or NULL.
+ *   flags W4A8_RELU | one W4A8_OUT_* | one W4A8_PATH_*.
+ *   Y     [M][ldy] out in the W4A8_OUT_* format, ldy >= N.
+ *   workspace: device memory of at least w4a8_workspace_size(M, K) bytes,
+ *       16-byte aligned; it holds the INT8 activations between kernels and
+ *       must not be touched by the caller until the call's work completes.
+ * M == 0 is a no-op returning W4A8_OK.
+ */
+W4A8_API w4a8_status w4a8_linear(const float *X, int M, int K, int ldx,
+                        const uint8_t *Wp, int ldp, const float *sw, int N,
+                        const float *bias, unsigned flags,
+                        void *Y, int ldy,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w4a8_linear_q - steps 4-6 on activations already quantized (by
+ * a8_quantize_rows or an equivalent producer).
+ *   Xq [M][ldq] int8 (ldq >= K, multiple of 16, 16-byte aligned), sx [M].
+ *   Bytes of Xq past K in a row may hold anything: they always meet zero
+ *   weight nibbles.
+ * Other arguments as for w4a8_linear. No workspace is needed.
+ */
+W4A8_API w4a8_status w4a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                          const uint8_t *Wp, int ldp, const float *sw, int N,
+                          const float *bias, unsigned flags,
+                          void *Y, int ldy, void *stream);
+
+/* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
+ * last successful w4a8_linear / w4a8_linear_q call enqueued; 0 if none. */
+W4A8_API unsigned w4a8_last_path(void);
+
+/* Read (and with clear != 0, reset) the current device's status word, which
+ * kernels set on an internal fault. Synchronizes `stream` first. */
+W4A8_API w4a8_status w4a8_get_device_status(int clear, void *stream);
+
+/* A static, human-readable name for a status code. */
+W4A8_API const char *w4a8_status_string(w4a8_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_H */

@@ -30,3 +30,17 @@ def read_golden(name: str) -> list[tuple[str, list[str]]]:
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+def pytest_sessionstart(session):
+    """Build the oracle (gcc) and libw4a8.so (nvcc, sm_100a) when stale, so a
+    fresh checkout tests what its sources say."""
+    import oracle
+    from w4a8_quantized_gemm_channel_b200 import build as native_build
+    oracle.build()
+    native_build.build()
+
+
+def cuda_ok() -> bool:
+    import torch
+    return torch.cuda.is_available()

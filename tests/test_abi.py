@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "w4a8.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return [n for n in re.findall(r"^W4A8_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, re.M)]
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    for must in ("w4_quantize_pack", "a8_quantize_rows", "w4a8_linear", "w4a8_linear_q",
+                 "w4a8_workspace_size", "w4a8_packed_ld", "w4a8_get_device_status",
+                 "w4a8_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from w4a8_quantized_gemm_channel_b200 import native
+    raw = ctypes.CDLL(native.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(raw, name), name
+        assert name in native.SIGNATURES, name
+
+
+def test_size_queries():
+    from w4a8_quantized_gemm_channel_b200 import native
+    import oracle
+    for k in (1, 2, 10, 31, 32, 33, 4096, 28672):
+        assert native.packed_ld(k) == oracle.packed_ld(k)
+        assert native.act_ld(k) % 16 == 0 and native.act_ld(k) >= k
+    assert native.packed_ld(0) == -1
+    assert native.workspace_size(0, 8) > 0
+    assert native.workspace_size(-1, 8) == 0
+    assert native.workspace_size(16, 4096) >= 16 * 4096 + 16 * 4
+
+
+def test_status_strings():
+    from w4a8_quantized_gemm_channel_b200 import native
+    for s in range(7):
+        assert native.lib.w4a8_status_string(s)
+    assert native.lib.w4a8_status_string(99) == b"unknown status"
+
+
+def _linear(lib, **kw):
+    a = dict(X=16, M=4, K=64, ldx=64, Wp=4096, ldp=32, sw=8192, N=8, bias=None, flags=0,
+             Y=12288, ldy=8, ws=16384, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.w4a8_linear(a["X"], a["M"], a["K"], a["ldx"], a["Wp"], a["ldp"], a["sw"], a["N"],
+                           a["bias"], a["flags"], a["Y"], a["ldy"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(K=0), 1), (dict(N=0), 1), (dict(M=-1), 1), (dict(K=2097153), 1),
+    (dict(ldp=16), 1),            # ldp < ceil(K/2)
+    (dict(ldp=40), 1),            # not a multiple of 16
+    (dict(Wp=4100), 1),           # Wp not 16-byte aligned
+    (dict(ldx=63), 1), (dict(ldy=7), 1),
+    (dict(Y=None), 1), (dict(sw=None), 1),
+    (dict(flags=0x04 | 0x01), 1),  # S32 output with ReLU
+    (dict(flags=0x04, bias=64), 1),  # S32 output with a bias
+    (dict(flags=0x06), 1),         # two output formats
+    (dict(flags=0x100), 1),        # unknown flag bit
+    (dict(ws=None), 3), (dict(wsb=10), 3), (dict(ws=16392), 3),
+    (dict(M=0), 0),                # no rows: a no-op
+])
+def test_linear_argument_checks(kw, want):
+    """Rejected before any device work (these run without a GPU)."""
+    from w4a8_quantized_gemm_channel_b200 import native
+    assert _linear(native.lib, **kw) == want
+
+
+def test_quantize_argument_checks():
+    from w4a8_quantized_gemm_channel_b200 import native
+    lib = native.lib
+    assert lib.w4_quantize_pack(16, 0, 8, 8, 4096, 16, 64, None) == 1
+    assert lib.w4_quantize_pack(16, 64, 8, 7, 4096, 32, 64, None) == 1   # ldw < N
+    assert lib.w4_quantize_pack(16, 64, 8, 8, 4096, 16, 64, None) == 1   # ldp too small
+    assert lib.w4_quantize_pack(16, 64, 8, 8, 4104, 32, 64, None) == 1   # Wp misaligned
+    assert lib.a8_quantize_rows(16, 0, 64, 64, 4096, 64, 64, None) == 0  # M = 0: no-op
+    assert lib.a8_quantize_rows(16, 2, 64, 64, 4096, 72, 64, None) == 1  # ldq % 16
+    assert lib.a8_quantize_rows(16, 2, 64, 60, 4096, 64, 64, None) == 1  # ldx < K
+    assert lib.w4a8_linear_q(24, 2, 64, 64, 64, 4096, 32, 64, 8, None, 0, 8192, 8, None) == 1  # Xq misaligned
+
+
+def test_no_device_means_unsupported_not_a_crash():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    from w4a8_quantized_gemm_channel_b200 import native
+    assert _linear(native.lib) == 2

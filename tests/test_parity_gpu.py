@@ -1,0 +1,294 @@
+"""GPU parity: every kernel path against the CPU oracle on the same seeded inputs.
+
+Bars (the layer's stated tolerances):
+  * packed weights, weight scales, INT8 activations, activation scales and the
+    INT32 accumulator: bit-exact;
+  * float32 output: |y - y_oracle| <= 1e-6 * |y_oracle| (with a bias,
+    1e-6 * (|y_oracle| + |b|), since a sum can cancel);
+  * bfloat16 output: within 1 bf16 ulp of the oracle's bf16 rounding.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w4a8_quantized_gemm_channel_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-6
+
+
+@pytest.fixture(scope="module")
+def nat():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from w4a8_quantized_gemm_channel_b200 import native
+    native.get_device_status(clear=True)
+    yield native
+    assert native.get_device_status() == 0, "a kernel recorded an internal fault"
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def assert_f32_close(y, ref, bias=None, rtol=RTOL):
+    y = np.asarray(y, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.abs(ref)
+    if bias is not None:
+        scale = scale + np.abs(np.asarray(bias, np.float64))[None, :]
+    bad = np.abs(y - ref) > rtol * scale
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outputs outside {rtol} relative"
+
+
+def assert_bf16_within_ulp(ybits, refbits):
+    a = np.asarray(ybits).view(np.int16).astype(np.int32)
+    b = np.asarray(refbits).view(np.int16).astype(np.int32)
+    assert (np.abs(a - b) <= 1).all()
+
+
+# ------------------------------------------------------------ weights ---
+
+@pytest.mark.parametrize("k,n", [(1, 1), (10, 32), (32, 1), (33, 7), (130, 45), (1152, 256),
+                                 (4096, 4096)])
+def test_quantize_pack_bit_exact(nat, k, n):
+    w = synth.linear_weights(k, n, 0.02, seed=100 + k + n)
+    if n > 2:
+        w[:, 1] = 0.0                      # an all-zero output channel
+    wp, sw = nat.w4_quantize_pack(dev(w))
+    wp_ref, sw_ref = oracle.w4_quantize_pack(w)
+    assert np.array_equal(host(sw).view(np.uint32), sw_ref.view(np.uint32))
+    assert np.array_equal(host(wp), wp_ref)
+
+
+def test_quantize_pack_wide_stride_and_padding(nat):
+    k, n = 77, 20
+    w = synth.linear_weights(k, 24, 0.02, seed=7)     # ldw = 24 > N
+    wd = dev(w)[:, :n]
+    ldp = 96                                         # more than ceil(77/2)
+    wp = torch.full((n, ldp), 0xAB, dtype=torch.uint8, device="cuda")
+    nat.w4_quantize_pack(wd, wp=wp)
+    wp_ref, _ = oracle.w4_quantize_pack(np.ascontiguousarray(w[:, :n]), ldp=ldp)
+    assert np.array_equal(host(wp), wp_ref)          # pad bytes overwritten with 0
+
+
+# -------------------------------------------------------- activations ---
+
+@pytest.mark.parametrize("m,k", [(1, 1), (32, 10), (3, 37), (16, 4096), (2048, 4096), (5, 6912)])
+def test_act_quant_bit_exact(nat, m, k):
+    x, _ = synth.linear_activations(m, k, seed=200 + m, outlier_count=min(8, k), outlier_factor=20.0)
+    if m > 2:
+        x[1] = 0.0                          # an all-zero row
+    xq, sx = nat.a8_quantize_rows(dev(x))
+    ldq = xq.shape[1]
+    xq_ref, sx_ref = oracle.a8_quantize_rows(x, ldq=ldq)
+    assert np.array_equal(host(sx).view(np.uint32), sx_ref.view(np.uint32))
+    assert np.array_equal(host(xq), xq_ref)
+
+
+def test_act_quant_unaligned_stride(nat):
+    x = synth.normal((9, 51), 1.0, synth.rng_for(3, 3))   # ldx = 51: no float4 loads
+    xd = dev(x)[:, 1:50]
+    xq, sx = nat.a8_quantize_rows(xd)
+    xq_ref, sx_ref = oracle.a8_quantize_rows(np.ascontiguousarray(x[:, 1:50]), ldq=xq.shape[1])
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(sx), sx_ref)
+
+
+def test_act_quant_empty(nat):
+    x = torch.empty((0, 64), device="cuda")
+    xq, sx = nat.a8_quantize_rows(x)
+    assert xq.shape[0] == 0 and sx.shape[0] == 0
+
+
+# ------------------------------------------------------------- linear ---
+
+PATHS = ["generic", "decode", "tc"]
+
+
+def _case(m, k, n, seed, outliers=4):
+    w = synth.linear_weights(k, n, 0.02, seed)
+    x, _ = synth.linear_activations(m, k, seed, outlier_count=min(outliers, k), outlier_factor=20.0)
+    b = synth.bias_vector(n, seed)
+    return x, w, b
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("m,k,n", [(1, 64, 16), (3, 33, 17), (8, 256, 40), (16, 4096, 64),
+                                   (17, 300, 33), (40, 1000, 130), (300, 520, 300),
+                                   (256, 4096, 1024)])
+def test_linear_s32_bit_exact(nat, path, m, k, n):
+    x, w, _ = _case(m, k, n, seed=300 + m + k + n)
+    wp, sw = oracle.w4_quantize_pack(w)
+    acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32", path=path)
+    assert nat.last_path() == path
+    assert np.array_equal(host(acc), oracle.linear(x, wp, sw, k, out="s32"))
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("relu", [False, True])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_linear_f32_and_bf16(nat, path, relu, with_bias):
+    m, k, n = 12, 520, 72
+    x, w, b = _case(m, k, n, seed=400 + relu + 2 * with_bias)
+    bias = b if with_bias else None
+    wp, sw = oracle.w4_quantize_pack(w)
+    args = (dev(x), dev(wp), dev(sw))
+    y = nat.w4a8_linear(*args, bias=None if bias is None else dev(bias), relu=relu, path=path)
+    ref = oracle.linear(x, wp, sw, k, bias=bias, relu=relu)
+    assert_f32_close(host(y), ref, bias)
+    if relu:
+        assert (host(y) >= 0).all()
+    yb = nat.w4a8_linear(*args, bias=None if bias is None else dev(bias), relu=relu,
+                         out="bf16", path=path)
+    refb = oracle.linear(x, wp, sw, k, bias=bias, relu=relu, out="bf16")
+    assert_bf16_within_ulp(host(yb.view(torch.int16)), refb)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_linear_q_matches_oracle_and_ignores_pad_bytes(nat, path):
+    m, k, n = 6, 100, 24
+    x, w, _ = _case(m, k, n, seed=500)
+    wp, sw = oracle.w4_quantize_pack(w)
+    xq_ref, sx_ref = oracle.a8_quantize_rows(x, ldq=112)
+    xq_dirty = xq_ref.copy()
+    xq_dirty[:, k:] = 77                      # garbage past K must not matter
+    y = nat.w4a8_linear_q(dev(xq_dirty), dev(sx_ref), k, dev(wp), dev(sw), path=path)
+    assert_f32_close(host(y), oracle.linear_q(xq_ref, sx_ref, wp, sw, k))
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_linear_output_stride_leaves_canaries(nat, path):
+    m, k, n = 5, 128, 20
+    x, w, _ = _case(m, k, n, seed=600)
+    wp, sw = oracle.w4_quantize_pack(w)
+    ybuf = torch.full((m + 1, 32), 12345.0, device="cuda")
+    y = ybuf[:m, :n]
+    nat.w4a8_linear(dev(x), dev(wp), dev(sw), y=y, path=path)
+    yb = host(ybuf)
+    assert (yb[:m, n:] == 12345.0).all() and (yb[m:] == 12345.0).all()
+    assert_f32_close(yb[:m, :n], oracle.linear(x, wp, sw, k))
+
+
+def test_linear_zero_rows_is_a_noop(nat):
+    wp = torch.zeros((8, 16), dtype=torch.uint8, device="cuda")
+    sw = torch.ones(8, device="cuda")
+    y = nat.w4a8_linear(torch.empty((0, 20), device="cuda"), wp, sw)
+    assert y.shape == (0, 8)
+
+
+def test_linear_zero_weight_column_gives_bias(nat):
+    m, k, n = 4, 64, 8
+    x, w, b = _case(m, k, n, seed=700)
+    w[:, 3] = 0.0
+    wpd, swd = nat.w4_quantize_pack(dev(w))
+    y = host(nat.w4a8_linear(dev(x), wpd, swd, bias=dev(b)))
+    assert (y[:, 3] == b[3]).all()
+
+
+# ------------------------------------------------- the minimal model ---
+
+def test_minimal_mlp_end_to_end(nat):
+    """The page's model: Dense(10->32, ReLU) -> Dense(32->1), both W4A8."""
+    d = synth.minimal_mlp(seed=0)
+    wp1, sw1 = nat.w4_quantize_pack(dev(d.w1))
+    wp2, sw2 = nat.w4_quantize_pack(dev(d.w2))
+    h = nat.w4a8_linear(dev(d.x), wp1, sw1, bias=dev(d.b1), relu=True)
+    y = host(nat.w4a8_linear(h, wp2, sw2, bias=dev(d.b2)))
+    ref = oracle.mlp(d.x, d.w1, d.b1, d.w2, d.b2)
+    assert np.array_equal(host(wp1), oracle.w4_quantize_pack(d.w1)[0])
+    assert_f32_close(y, ref)
+    x64 = d.x.astype(np.float64)
+    yfp = np.maximum(x64 @ d.w1 + d.b1, 0) @ d.w2 + d.b2
+    mse = float(np.mean((yfp - y) ** 2))
+    assert 0 < mse <= 1e-2
+
+
+def test_determinism(nat):
+    m, k, n = 16, 4096, 512
+    x, w, _ = _case(m, k, n, seed=800)
+    wpd, swd = nat.w4_quantize_pack(dev(w))
+    xd = dev(x)
+    a = host(nat.w4a8_linear(xd, wpd, swd))
+    b = host(nat.w4a8_linear(xd, wpd, swd))
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+# --------------------------------------------- full-size workloads ---
+
+@pytest.mark.parametrize("m", synth.DECODE_MS)
+def test_decode_full_size(nat, m):
+    """Decode single linear at full size (K = N = 4096), auto dispatch - the
+    configuration the benchmark times - checked on every output."""
+    c = synth.decode_case(m)
+    wpd, swd = nat.w4_quantize_pack(dev(c.w))
+    wp, sw = oracle.w4_quantize_pack(c.w)
+    assert np.array_equal(host(wpd), wp)
+    y = nat.w4a8_linear(dev(c.x), wpd, swd)
+    assert_f32_close(host(y), oracle.linear(c.x, wp, sw, synth.DECODE_K))
+    acc = nat.w4a8_linear(dev(c.x), wpd, swd, out="s32")
+    assert np.array_equal(host(acc), oracle.linear(c.x, wp, sw, synth.DECODE_K, out="s32"))
+
+
+def _sampled_check(nat, x, w, wpd, swd, rows, cols, relu=False, path="auto"):
+    """Full-size run on the GPU; the oracle recomputes sampled rows x channels
+    (each sampled row is quantized over its full K)."""
+    wp_ref, sw_ref = oracle.w4_quantize_pack(w[:, cols]) if w is not None else (None, None)
+    y = host(nat.w4a8_linear(dev(x), wpd, swd, relu=relu, path=path))
+    wp_s = host(wpd)[cols]
+    sw_s = host(swd)[cols]
+    if wp_ref is not None:
+        assert np.array_equal(wp_s, wp_ref)
+        assert np.array_equal(sw_s, sw_ref)
+    ref = oracle.linear(x[rows], wp_s, sw_s, x.shape[1], relu=relu)
+    assert_f32_close(y[np.ix_(rows, cols)], ref)
+    return y
+
+
+def test_gemma_stack_shapes_sampled(nat):
+    """One layer of the Gemma3-1B-shaped stack at M = 1 and M = 512."""
+    rng = synth.rng_for(9, 9)
+    for p, (name, k, n) in enumerate(synth.GEMMA_PROJ):
+        w = synth.gemma_weights(0, p)
+        wpd, swd = nat.w4_quantize_pack(dev(w))
+        for m in synth.GEMMA_MS:
+            x = synth.gemma_activations(m, k, sub=p)
+            rows = np.unique(rng.integers(0, m, size=min(m, 8)))
+            cols = np.unique(rng.integers(0, n, size=48))
+            _sampled_check(nat, x, w, wpd, swd, rows, cols)
+
+
+def test_prefill_full_size_sampled(nat):
+    """Prefill single linear at full size (M=2048, K=4096, N=11008), plain and
+    with the fused ReLU; sampled rows x channels recomputed by the oracle."""
+    c = synth.prefill_case()
+    wpd, swd = nat.w4_quantize_pack(dev(c.w))
+    rng = synth.rng_for(10, 10)
+    rows = np.unique(np.concatenate([[0, 2047], rng.integers(0, 2048, size=6)]))
+    cols = np.unique(np.concatenate([[0, 11007], rng.integers(0, 11008, size=60)]))
+    for relu in (False, True):
+        _sampled_check(nat, c.x, c.w, wpd, swd, rows, cols, relu=relu)
+
+
+@pytest.mark.parametrize("shape", [0, 1])
+def test_llama70_shapes_sampled(nat, shape):
+    """70B-shaped linears at full size for M in {1, 16, 128, 4096}."""
+    c0 = synth.llama70_case(shape, 1, with_x=False)
+    k, n = synth.LLAMA70_SHAPES[shape]
+    wpd, swd = nat.w4_quantize_pack(dev(c0.w))
+    rng = synth.rng_for(11, shape)
+    cols = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, size=40)]))
+    wp_ref, sw_ref = oracle.w4_quantize_pack(c0.w[:, cols])
+    assert np.array_equal(host(wpd)[cols], wp_ref)
+    assert np.array_equal(host(swd)[cols], sw_ref)
+    for m in synth.LLAMA70_MS:
+        c = synth.llama70_case(shape, m)
+        rows = np.unique(np.concatenate([[0, m - 1], rng.integers(0, m, size=4)]))
+        _sampled_check(nat, c.x, None, wpd, swd, rows, cols)

@@ -1,0 +1,84 @@
+// Shared device helpers of libw4a8 (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "w4a8.h"
+
+namespace w4a8 {
+
+// One status word per device. Kernels record the first internal fault here
+// (bounds or a bounded wait that ran out) instead of trapping, so the context
+// stays usable and the host can read the code back. The library is one
+// translation unit (w4a8_abi.cu includes every kernel header), so this is the
+// only definition.
+__device__ int g_device_status = 0;
+
+__device__ __forceinline__ void record_fault(int code) {
+    atomicCAS(&g_device_status, 0, code);
+}
+
+// Programmatic dependent launch: wait for the grids this one depends on to
+// finish (their writes are then visible), and let dependents start launching.
+// Both are no-ops when the launch carries no programmatic dependency.
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Warm L2 with [p, p + bytes) (bytes a multiple of 16, p 16-byte aligned)
+// without returning data: safe to issue before griddepcontrol.wait, because
+// L2 is the point of coherence and no stale value reaches a register.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Sign-extend the eight 4-bit two's-complement codes of one packed word.
+// Byte b of `p` holds codes k = 2b (low nibble) and k = 2b + 1 (high nibble).
+// Returns lo = bytes {k0, k2, k4, k6} and hi = bytes {k1, k3, k5, k7} as INT8.
+// Nibble v becomes v | 0xF0 when its sign bit (bit 3) is set: the product
+// (bit3 << 3) * 0x1E = 0xF0 stays inside its byte, so one multiply sets the
+// high nibbles of all four bytes at once.
+__device__ __forceinline__ void unpack_s4x8(uint32_t p, uint32_t &lo, uint32_t &hi) {
+    const uint32_t m = 0x0F0F0F0Fu, s = 0x08080808u;
+    uint32_t t = p >> 4;
+    lo = (p & m) + (p & s) * 0x1Eu;
+    hi = (t & m) + (t & s) * 0x1Eu;
+}
+
+// Dequantize one INT32 accumulator and apply the Dense epilogue, in the same
+// float32 operations and order as the method's statement:
+//   y = float(acc) / (sx * sw); y += bias; y = y > 0 ? y : +0.
+__device__ __forceinline__ float dequant_one(int32_t acc, float sxm, float swn,
+                                             const float *__restrict__ bias, int n,
+                                             bool relu) {
+    float d = __fmul_rn(sxm, swn);
+    float y = __fdiv_rn(__int2float_rn(acc), d);
+    if (bias) y = __fadd_rn(y, bias[n]);
+    if (relu) y = y > 0.0f ? y : 0.0f;
+    return y;
+}
+
+__device__ __forceinline__ void store_out(void *__restrict__ Y, int ldy, int m, int n,
+                                          int32_t acc, float sxm, float swn,
+                                          const float *__restrict__ bias, unsigned flags) {
+    size_t off = (size_t)m * (size_t)ldy + (size_t)n;
+    unsigned fmt = flags & W4A8_OUT_MASK;
+    if (fmt == W4A8_OUT_S32) {
+        static_cast<int32_t *>(Y)[off] = acc;
+        return;
+    }
+    float y = dequant_one(acc, sxm, swn, bias, n, (flags & W4A8_RELU) != 0);
+    if (fmt == W4A8_OUT_BF16)
+        static_cast<__nv_bfloat16 *>(Y)[off] = __float2bfloat16_rn(y);
+    else
+        static_cast<float *>(Y)[off] = y;
+}
+
+__device__ __forceinline__ int clampi(int v, int lo, int hi) { return min(max(v, lo), hi); }
+
+}  // namespace w4a8

@@ -1,0 +1,355 @@
+// Tensor-core path of the quantized product on sm_100a (steps 4-6 of "How it
+// works" in the Keras guide "INT4 quantization in Keras"): packed INT4 weights
+// are unpacked to INT8 on chip and multiplied with INT8 activations by
+// tcgen05.mma kind::i8, accumulating in INT32 in tensor memory (TMEM); the
+// epilogue dequantizes acc / (sx * sw) and applies bias and ReLU.
+//
+// The product is computed transposed, D^T[n][m] = sum_k q[n][k] * xq[m][k]:
+//  * A (M_mma = 128 output channels x K) comes from TMEM. A warpgroup reads the
+//    packed tile that TMA put in shared memory, sign-extends the nibbles in
+//    registers and writes the INT8 rows into TMEM with tcgen05.st, so the
+//    unpacked weights never travel through shared memory.
+//  * B (N_mma = BT tokens x K) is the INT8 activation tile, loaded by TMA with
+//    128-byte swizzling and read by the MMA through a shared-memory descriptor.
+//  * D lives in TMEM with output channels on lanes and tokens on columns, so
+//    an epilogue thread owns one output channel (one weight scale, one bias)
+//    and a warp stores 32 consecutive channels of a token row at once.
+//
+// One persistent CTA per SM walks the (channel tile, token tile) grid.
+// Warp roles (12 warps): warp 0 issues TMA loads, warp 1 owns TMEM and
+// issues the MMAs, warps 4-7 unpack weights, warps 8-11 run the epilogue.
+// Shared-memory stages and TMEM A slots form a STAGES-deep ring; the
+// accumulator is double-buffered so the epilogue of one tile overlaps the
+// main loop of the next. Every mbarrier wait is bounded (see ptx::mbar_wait).
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace w4a8 {
+namespace tc {
+
+constexpr int BM = 128;            // output channels per tile (MMA M)
+constexpr int BK = 128;            // k per stage
+constexpr int MMA_K = 32;          // k per kind::i8 instruction
+// 6 stages: 144 KB of shared memory, which also keeps a second CTA (that
+// would block in tcgen05.alloc of the whole TMEM) off the SM.
+constexpr int STAGES = 6;
+constexpr int NUM_THREADS = 384;
+constexpr int TMEM_COLS = 512;
+constexpr int A_COLS = BK / 4;     // TMEM columns per A slot (4 INT8 per column)
+constexpr int W_TILE_BYTES = BM * BK / 2;
+
+template <int BT>
+struct alignas(1024) Smem {
+    uint8_t act[STAGES][BT * BK];        // activation tiles, 128B-swizzled rows
+    uint8_t wpk[STAGES][W_TILE_BYTES];   // packed weight tiles, 64B-swizzled rows
+    uint64_t full[STAGES];               // TMA landed (tx-count barrier)
+    uint64_t aready[STAGES];             // A slot written to TMEM (4 unpack warps)
+    uint64_t empty[STAGES];              // MMAs reading the stage finished
+    uint64_t acc_full[2];                // accumulator ready for the epilogue
+    uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
+    uint64_t mma_done;                   // final drain of the MMA pipe
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <int BT>
+constexpr int d_col(int buf) { return buf * BT; }
+template <int BT>
+constexpr int a_col(int stage) { return 2 * BT + stage * A_COLS; }
+
+template <int BT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+          int M, int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
+          const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+    static_assert(2 * BT + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
+    extern __shared__ uint8_t smem_raw[];
+    Smem<BT> &sm = *reinterpret_cast<Smem<BT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_kb = (K + BK - 1) / BK;
+    const int tiles_m = (M + BT - 1) / BT;
+    const int tiles_n = (N + BM - 1) / BM;
+    const int num_tiles = tiles_m * tiles_n;
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&sm.full[s], 1);
+            ptx::mbar_init(&sm.aready[s], 4);
+            ptx::mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&sm.acc_full[b], 1);
+            ptx::mbar_init(&sm.acc_empty[b], 4);
+        }
+        ptx::mbar_init(&sm.mma_done, 1);
+        sm.abort = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tensormap(&tm_w);
+        ptx::prefetch_tensormap(&tm_x);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&sm.tmem_base, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    // Dependents may launch once every CTA of this grid is resident; the
+    // activations and scales come from the previous kernel, so wait for it.
+    griddep_launch_dependents();
+    griddep_wait();
+
+    if (warp == 0) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0;  // bit s: stage s has a load whose landing we have not seen
+            uint32_t last_par = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int n_tile = tile / tiles_m, m_tile = tile % tiles_m;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!ptx::mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&sm.full[stage], BT * BK + W_TILE_BYTES);
+                    ptx::tma_load_2d(sm.wpk[stage], &tm_w, kb * (BK / 2), n_tile * BM, &sm.full[stage]);
+                    ptx::tma_load_2d(sm.act[stage], &tm_x, kb * BK, m_tile * BT, &sm.full[stage]);
+                    issued |= 1u << stage;
+                    last_par = (last_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                // Drain: every load this thread issued lands before the CTA exits.
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued & (1u << s)) ptx::mbar_wait_drain(&sm.full[s], (last_par >> s) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_i8(BM, BT);
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true, any = false;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!ptx::mbar_wait(&sm.acc_empty[buf], acc_phase ^ 1, abort)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)d_col<BT>(buf);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!ptx::mbar_wait(&sm.full[stage], phase, abort) ||
+                        !ptx::mbar_wait(&sm.aready[stage], phase, abort)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t a = tmem + (uint32_t)a_col<BT>(stage);
+                    const uint32_t b = ptx::smem_addr(sm.act[stage]);
+#pragma unroll
+                    for (int kk = 0; kk < BK / MMA_K; ++kk) {
+                        ptx::mma_i8_ts(d, a + kk * (MMA_K / 4), ptx::sdesc_k_sw128(b + kk * MMA_K), idesc,
+                                       (kb | kk) != 0);
+                    }
+                    any = true;
+                    ptx::mma_commit(&sm.empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&sm.acc_full[buf]);
+                if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+            }
+            if (any) {
+                // All MMAs done before TMEM is released.
+                ptx::mma_commit(&sm.mma_done);
+                ptx::mbar_wait_drain(&sm.mma_done, 0);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------------------------------------------- weight unpack
+        // Thread r owns output-channel row r of the tile: 64 packed bytes per
+        // stage, read from the 64B-swizzled tile (16-byte chunk c of row r
+        // sits at chunk c ^ ((r >> 1) & 3)), expanded to 128 INT8 in k order
+        // and stored to TMEM lane r, 32 columns.
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                // every lane waits (each then sees the TMA data); the outcome is
+                // made warp-uniform before the warp-collective tcgen05.st
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sm.full[stage], phase, abort));
+                if (!ok) break;
+                const uint8_t *row = sm.wpk[stage] + r * (BK / 2);
+                const int sx_ = (r >> 1) & 3;
+                uint32_t out[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * (c ^ sx_));
+                    const uint32_t p[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t lo, hi;
+                        unpack_s4x8(p[j], lo, hi);  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
+                        out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
+                        out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                    }
+                }
+                ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)a_col<BT>(stage), out);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&sm.aready[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
+    } else if (warp >= 8) {
+        // ---------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        const unsigned fmt = flags & W4A8_OUT_MASK;
+        const bool relu = (flags & W4A8_RELU) != 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int n_tile = tile / tiles_m, m_tile = tile % tiles_m;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sm.acc_full[buf], acc_phase, abort))) break;
+            ptx::tc_fence_after();
+            const int n = n_tile * BM + q * 32 + lane;
+            const bool n_ok = n < N;
+            const float swn = n_ok ? __ldg(sw + n) : 1.0f;
+            const float bn = (bias && n_ok) ? __ldg(bias + n) : 0.0f;
+            const int m_base = m_tile * BT;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BT; c0 += 32) {
+                uint32_t v[32];
+                ptx::tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(d_col<BT>(buf) + c0), v);
+                ptx::tmem_wait_ld();
+                const int mrem = M - (m_base + c0);
+                if (mrem <= 0) break;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if (j < mrem && n_ok) {
+                        const int m = m_base + c0 + j;
+                        const size_t off = (size_t)m * (size_t)ldy + (size_t)n;
+                        const int32_t acc = (int32_t)v[j];
+                        if (fmt == W4A8_OUT_S32) {
+                            static_cast<int32_t *>(Y)[off] = acc;
+                        } else {
+                            float y = __fdiv_rn(__int2float_rn(acc), __fmul_rn(__ldg(sx + m), swn));
+                            if (bias) y = __fadd_rn(y, bn);
+                            if (relu) y = y > 0.0f ? y : 0.0f;
+                            if (fmt == W4A8_OUT_BF16)
+                                static_cast<__nv_bfloat16 *>(Y)[off] = __float2bfloat16_rn(y);
+                            else
+                                static_cast<float *>(Y)[off] = y;
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sm.acc_empty[buf]);
+            if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------- host side ---
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A 2-D byte tensor [rows][inner] with the given row stride; tiles of
+// box_inner bytes x box_rows rows; out-of-range elements read as zero.
+inline bool make_map_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows, uint64_t stride,
+                        uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {stride};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BT>
+inline size_t smem_bytes() { return sizeof(Smem<BT>) + 1024; }
+
+template <int BT>
+inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
+                          const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy, int sm_count,
+                          cudaStream_t stream) {
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(k_gemm_tc<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)smem_bytes<BT>());
+    });
+    if (attr_err != cudaSuccess) return W4A8_ERR_CUDA;
+    CUtensorMap tm_w, tm_x;
+    if (!make_map_u8(&tm_w, Wp, (uint64_t)ldp, (uint64_t)N, (uint64_t)ldp, BK / 2, BM,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_u8(&tm_x, Xq, (uint64_t)ldq, (uint64_t)M, (uint64_t)ldq, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return W4A8_ERR_CUDA;
+    const long long tiles = (long long)((M + BT - 1) / BT) * ((N + BM - 1) / BM);
+    const int grid = (int)(tiles < sm_count ? tiles : sm_count);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem_bytes<BT>();
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_tc<BT>, tm_w, tm_x, M, N, K, sx, sw, bias, flags, Y, ldy);
+    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
+}  // namespace tc
+
+inline bool tc_supported(int M, int K, int N) {
+    return M >= 1 && K >= 1 && N >= 1 && tc::encode_fn() != nullptr;
+}
+
+inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp,
+                                  int ldp, const float *sw, int N, const float *bias, unsigned flags, void *Y,
+                                  int ldy, int sm_count, cudaStream_t stream) {
+    return tc::launch<128>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+}
+
+}  // namespace w4a8

@@ -1,0 +1,186 @@
+// CUDA-core paths of the quantized product (steps 4-6 of "How it works" in the
+// Keras guide "INT4 quantization in Keras"): unpack INT4 -> INT8, INT8 x INT8
+// accumulated in INT32, dequantize acc / (sx * sw), bias, ReLU.
+//
+//  * k_linear_generic: one thread per output, any shape; used for tiny layers.
+//  * k_linear_decode : few activation rows (<= 16 per tile). The layer is then
+//    bound by streaming the packed weights from HBM, so each warp issues its
+//    16-byte weight loads up front and reduces them on the legacy integer
+//    tensor-core path (mma.sync m16n8k32 s8): the FLOPs are tiny, what matters
+//    is bytes in flight and few instructions per weight byte.
+#pragma once
+
+#include "common.cuh"
+
+namespace w4a8 {
+
+// ---------------------------------------------------------------------------
+// Generic kernel. grid = (ceil(N/128), min(M, 65535)), block = 128.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
+                 const float *__restrict__ sx,
+                 const uint8_t *__restrict__ Wp, int ldp, const float *__restrict__ sw, int N,
+                 const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    const uint8_t *wr = Wp + (size_t)n * ldp;
+    const float swn = __ldg(sw + n);
+    for (int m = blockIdx.y; m < M; m += gridDim.y) {
+        const int8_t *xr = Xq + (size_t)m * ldq;
+        int32_t acc = 0;
+        for (int k = 0; k < K; ++k) {
+            const uint32_t b = __ldg(wr + (k >> 1));
+            const int v = (k & 1) ? (int)(b >> 4) : (int)(b & 0xFu);
+            acc += (int32_t)__ldg(xr + k) * ((v ^ 8) - 8);
+        }
+        store_out(Y, ldy, m, n, acc, __ldg(sx + m), swn, bias, flags);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Decode kernel.
+//
+// Block = 8 warps = one 16-channel row block of the weight matrix; warp w owns
+// the 128-k chunks c = w, w+8, w+16, ... of K, so the block's warps read 512
+// contiguous bytes of each weight row between them. blockIdx.y selects a tile
+// of 8*NTG activation rows (tokens).
+//
+// mma.sync.m16n8k32 (A 16x32 row-major, B 32x8 col-major, s8 -> s32) with the
+// weights as A and the tokens as B. The dot product does not care which
+// physical k sits in which of the instruction's 32 k-slots, as long as A and B
+// agree. Thread (g = lane/4, t = lane%4) loads 16 bytes of weight rows g and
+// g+8 per chunk: bytes [64c + 16t, +16) = k in [128c + 32t, +32). Word j of
+// them (k = 128c + 32t + 8j .. +7) feeds MMA j: its low nibbles (even k) go to
+// A slots 4t..4t+3 and its high nibbles (odd k) to slots 16+4t..16+4t+3. The
+// B fragment of the same thread covers the same slots, so it takes the even
+// and odd bytes of xq[token][128c + 32t + 8j .. +7].
+//
+// PDL: before griddepcontrol.wait the block only asks for its 16 weight rows
+// to be brought into L2 (one bulk prefetch), so the HBM stream starts while
+// the activation-quantization kernel still runs, and every value the kernel
+// computes with is loaded after the wait.
+// ---------------------------------------------------------------------------
+constexpr int DEC_WARPS = 8;
+// chunks per warp per batch of loads: 4 for one token group, 2 for two (the
+// activation fragments double), which keeps two blocks per SM
+template <int NTG>
+constexpr int dec_unroll() { return NTG == 1 ? 4 : 2; }
+
+__device__ __forceinline__ void mma_s8_16832(int32_t (&c)[4], uint32_t a0, uint32_t a1,
+                                             uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int NTG>
+__global__ void __launch_bounds__(DEC_WARPS * 32)
+k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
+                const float *__restrict__ sx,
+                const uint8_t *__restrict__ Wp, int ldp, const float *__restrict__ sw, int N,
+                const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+    constexpr int TOK = 8 * NTG;
+    constexpr int DEC_UNROLL = dec_unroll<NTG>();
+    static_assert(16 * TOK <= DEC_WARPS * 32, "one epilogue element per thread");
+    __shared__ int32_t red[DEC_WARPS][16][TOK + 1];
+    griddep_launch_dependents();  // see k_act_quant: dependents only prefetch weights
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int n0 = blockIdx.x * 16;
+    const int m0 = blockIdx.y * TOK;
+    const int nchunks = (ldp + 63) / 64;  // 128-k chunks covering the packed rows
+
+    if (threadIdx.x == 0) {
+        const int rows = min(16, N - n0);
+        prefetch_l2_bulk(Wp + (size_t)n0 * ldp, (uint32_t)(rows * ldp));
+    }
+    griddep_wait();
+
+    // Epilogue operands, fetched now so their latency hides under the stream:
+    // thread e finishes output (channel n0 + e % 16, token m0 + e / 16).
+    const int e_ch = threadIdx.x % 16, e_tk = threadIdx.x / 16;
+    const bool e_ok = threadIdx.x < 16 * TOK && n0 + e_ch < N && m0 + e_tk < M;
+    float e_sw = 1.0f, e_sx = 1.0f;
+    if (e_ok) {
+        e_sw = __ldg(sw + n0 + e_ch);
+        e_sx = __ldg(sx + m0 + e_tk);
+    }
+
+    const bool row_lo_ok = n0 + g < N, row_hi_ok = n0 + g + 8 < N;
+    const uint8_t *wlo = Wp + (size_t)(row_lo_ok ? n0 + g : 0) * ldp + 16 * t;
+    const uint8_t *whi = Wp + (size_t)(row_hi_ok ? n0 + g + 8 : 0) * ldp + 16 * t;
+
+    int32_t acc[NTG][4];
+#pragma unroll
+    for (int i = 0; i < NTG; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0;
+
+    for (int cb = warp; cb < nchunks; cb += DEC_WARPS * DEC_UNROLL) {
+        // Issue every load of this batch before any use: weights and the
+        // matching INT8 activations (an out-of-range piece reads as zeros).
+        uint4 wa[DEC_UNROLL], wb[DEC_UNROLL], xv[DEC_UNROLL][NTG][2];
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {
+            const int c = cb + u * DEC_WARPS;
+            const int off = 64 * c;                // this thread's piece: off + 16t
+            const bool in = c < nchunks && off + 16 * t < ldp;
+            wa[u] = (in && row_lo_ok) ? __ldg(reinterpret_cast<const uint4 *>(wlo + off)) : make_uint4(0, 0, 0, 0);
+            wb[u] = (in && row_hi_ok) ? __ldg(reinterpret_cast<const uint4 *>(whi + off)) : make_uint4(0, 0, 0, 0);
+            const int kbase = 128 * c + 32 * t;
+#pragma unroll
+            for (int i = 0; i < NTG; ++i) {
+                const int m = m0 + 8 * i + g;
+                const int8_t *xr = Xq + (size_t)m * ldq + kbase;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const bool ok = c < nchunks && m < M && kbase + 16 * h < ldq;
+                    xv[u][i][h] = ok ? __ldg(reinterpret_cast<const uint4 *>(xr + 16 * h)) : make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {
+            if (cb + u * DEC_WARPS >= nchunks) continue;  // warp-uniform
+            const uint32_t pa[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
+            const uint32_t pb[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t alo, ahi, blo, bhi;
+                unpack_s4x8(pa[j], alo, ahi);
+                unpack_s4x8(pb[j], blo, bhi);
+#pragma unroll
+                for (int i = 0; i < NTG; ++i) {
+                    const uint4 &v = xv[u][i][j >> 1];
+                    const uint32_t x0 = (j & 1) ? v.z : v.x;
+                    const uint32_t x1 = (j & 1) ? v.w : v.y;
+                    const uint32_t b0 = __byte_perm(x0, x1, 0x6420);  // even k
+                    const uint32_t b1 = __byte_perm(x0, x1, 0x7531);  // odd k
+                    mma_s8_16832(acc[i], alo, blo, ahi, bhi, b0, b1);
+                }
+            }
+        }
+    }
+
+    // C fragment: rows g, g+8 (channels), columns 2t, 2t+1 (tokens).
+#pragma unroll
+    for (int i = 0; i < NTG; ++i) {
+        red[warp][g][8 * i + 2 * t] = acc[i][0];
+        red[warp][g][8 * i + 2 * t + 1] = acc[i][1];
+        red[warp][g + 8][8 * i + 2 * t] = acc[i][2];
+        red[warp][g + 8][8 * i + 2 * t + 1] = acc[i][3];
+    }
+    __syncthreads();
+    if (e_ok) {
+        int32_t s = 0;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) s += red[w][e_ch][e_tk];
+        store_out(Y, ldy, m0 + e_tk, n0 + e_ch, s, e_sx, e_sw, bias, flags);
+    }
+}
+
+}  // namespace w4a8

@@ -1,0 +1,280 @@
+// extern "C" entry points of libw4a8.so: argument checks, workspace layout,
+// kernel selection and launches. Declarations and contracts: include/w4a8.h.
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "w4a8.h"
+#include "common.cuh"
+#include "quant_kernels.cuh"
+#include "linear_simt.cuh"
+#include "gemm_tc.cuh"
+
+namespace w4a8 {
+namespace {
+
+thread_local unsigned t_last_path = 0;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0;
+    bool ok = false;
+};
+
+// Per-device properties, read once per device.
+const DeviceInfo &device_info() {
+    static std::mutex mu;
+    static DeviceInfo infos[64];
+    static bool done[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        static DeviceInfo none;
+        return none;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess)
+            d.ok = (d.major == 10);
+        infos[dev] = d;
+        done[dev] = true;
+    }
+    return infos[dev];
+}
+
+// Launch with the programmatic-stream-serialization attribute, so a kernel
+// may begin its prologue while its predecessor in the stream finishes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+w4a8_status from_cuda(cudaError_t e) { return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA; }
+
+struct Workspace {
+    int8_t *xq;
+    float *sx;
+    int ldq;
+};
+
+size_t workspace_bytes_for(int M, int K, int *ldq_out) {
+    const int ldq = round_up(K, 16);
+    if (ldq_out) *ldq_out = ldq;
+    const size_t xq_bytes = ((size_t)M * (size_t)ldq + 255) / 256 * 256;
+    return xq_bytes + (size_t)M * sizeof(float) + 256;
+}
+
+Workspace carve_workspace(void *ws, int M, int K) {
+    Workspace w;
+    workspace_bytes_for(M, K, &w.ldq);
+    uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + 255) & ~uintptr_t(255);
+    w.xq = reinterpret_cast<int8_t *>(base);
+    base += ((size_t)M * (size_t)w.ldq + 255) / 256 * 256;
+    w.sx = reinterpret_cast<float *>(base);
+    return w;
+}
+
+w4a8_status check_common(int M, int K, int N, const uint8_t *Wp, int ldp, const float *sw,
+                         const float *bias, unsigned flags, const void *Y, int ldy) {
+    if (K < 1 || K > W4A8_MAX_K || N < 1 || M < 0) return W4A8_ERR_INVALID_ARG;
+    if (!Wp || !sw || (!Y && M > 0)) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(Wp) || ldp < (K + 1) / 2 || ldp % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (ldy < N || !aligned4(sw) || (bias && !aligned4(bias))) return W4A8_ERR_INVALID_ARG;
+    const unsigned fmt = flags & W4A8_OUT_MASK;
+    if (fmt == (W4A8_OUT_BF16 | W4A8_OUT_S32)) return W4A8_ERR_INVALID_ARG;
+    if (fmt == W4A8_OUT_S32 && (bias || (flags & W4A8_RELU))) return W4A8_ERR_INVALID_ARG;
+    const size_t esz = fmt == W4A8_OUT_BF16 ? 2 : 4;
+    if ((reinterpret_cast<uintptr_t>(Y) & (esz - 1)) != 0) return W4A8_ERR_INVALID_ARG;
+    if (flags & ~(W4A8_RELU | W4A8_OUT_MASK | W4A8_PATH_MASK)) return W4A8_ERR_INVALID_ARG;
+    return W4A8_OK;
+}
+
+// Kernel selection by shape. Few rows: the layer is a weight stream, so the
+// decode kernel; many rows: the tensor-core GEMM; tiny problems: generic.
+unsigned choose_path(int M, int K, int N, unsigned flags) {
+    const unsigned forced = flags & W4A8_PATH_MASK;
+    if (forced) return forced;
+    const double work = (double)M * (double)N * (double)K;
+    if (work < 65536.0) return W4A8_PATH_GENERIC;
+    if (M <= 16) return W4A8_PATH_DECODE;
+    if (tc_supported(M, K, N)) return W4A8_PATH_TC;
+    return W4A8_PATH_DECODE;
+}
+
+w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                        const uint8_t *Wp, int ldp, const float *sw, int N,
+                        const float *bias, unsigned flags, void *Y, int ldy,
+                        cudaStream_t stream) {
+    const DeviceInfo &dev = device_info();
+    if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
+    const unsigned path = choose_path(M, K, N, flags);
+    cudaError_t e = cudaSuccess;
+    if (path == W4A8_PATH_GENERIC) {
+        dim3 grid((N + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
+        e = launch_pdl(k_linear_generic, grid, dim3(128), 0, stream,
+                       Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+    } else if (path == W4A8_PATH_DECODE) {
+        const int tok = M <= 8 ? 8 : 16;
+        const int tiles = (M + tok - 1) / tok;
+        if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
+        dim3 grid((N + 15) / 16, tiles);
+        if (tok == 8)
+            e = launch_pdl(k_linear_decode<1>, grid, dim3(DEC_WARPS * 32), 0, stream,
+                           Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+        else
+            e = launch_pdl(k_linear_decode<2>, grid, dim3(DEC_WARPS * 32), 0, stream,
+                           Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+    } else if (path == W4A8_PATH_TC) {
+        if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
+        w4a8_status st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+                                        dev.sm_count, stream);
+        if (st != W4A8_OK) return st;
+    } else {
+        return W4A8_ERR_INVALID_ARG;
+    }
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    t_last_path = path;
+    return W4A8_OK;
+}
+
+}  // namespace
+}  // namespace w4a8
+
+using namespace w4a8;
+
+extern "C" {
+
+int w4a8_packed_ld(int K) { return K < 1 ? -1 : round_up((K + 1) / 2, 16); }
+
+int w4a8_act_ld(int K) { return K < 1 ? -1 : round_up(K, 16); }
+
+size_t w4a8_workspace_size(int M, int K) {
+    if (M < 0 || K < 1) return 0;
+    return workspace_bytes_for(M, K, nullptr);
+}
+
+w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp, int ldp,
+                             float *sw, void *stream) {
+    if (!W || !Wp || !sw || K < 1 || K > W4A8_MAX_K || N < 1 || ldw < N) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(Wp) || ldp < (K + 1) / 2 || ldp % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (!aligned4(W) || !aligned4(sw)) return W4A8_ERR_INVALID_ARG;
+    const DeviceInfo &dev = device_info();
+    if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned *amax = reinterpret_cast<unsigned *>(sw);
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * (size_t)N, s);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    // K-slices so that the abs-max pass puts a few blocks on every SM.
+    const int col_blocks = (N + 31) / 32;
+    int splits = (4 * dev.sm_count + col_blocks - 1) / col_blocks;
+    splits = splits < 1 ? 1 : splits;
+    int rows = (K + splits - 1) / splits;
+    rows = round_up(rows < 64 ? 64 : rows, 8);
+    splits = (K + rows - 1) / rows;
+    k_col_absmax<<<dim3(col_blocks, splits), dim3(32, 8), 0, s>>>(W, K, N, ldw, rows, amax);
+    if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
+    const int kblocks = (2 * ldp + 63) / 64;
+    if (kblocks > 65535) return W4A8_ERR_UNSUPPORTED;
+    k_quant_pack<<<dim3(col_blocks, kblocks), dim3(32, 8), 0, s>>>(W, K, N, ldw, amax, Wp, ldp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
+    k_weight_scale_finalize<<<(N + 255) / 256, 256, 0, s>>>(sw, N);
+    return from_cuda(cudaGetLastError());
+}
+
+static w4a8_status launch_act_quant(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
+                                    float *sx, cudaStream_t s) {
+    const int vec4 = aligned16(X) && (ldx % 4 == 0);
+    const int grid = M < 65535 ? M : 65535;
+    cudaError_t e;
+    if (K <= 1024)
+        e = launch_pdl(k_act_quant<128, 8>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+    else
+        e = launch_pdl(k_act_quant<256, 16>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+    return from_cuda(e);
+}
+
+w4a8_status a8_quantize_rows(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
+                             float *sx, void *stream) {
+    if (M < 0 || K < 1 || K > W4A8_MAX_K || ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (ldq < K || ldq % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || !Xq || !sx || !aligned16(Xq) || !aligned4(X) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    return launch_act_quant(X, M, K, ldx, Xq, ldq, sx, static_cast<cudaStream_t>(stream));
+}
+
+w4a8_status w4a8_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp,
+                        const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    if (workspace_bytes < w4a8_workspace_size(M, K)) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    const Workspace ws = carve_workspace(workspace, M, K);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
+    if (st != W4A8_OK) return st;
+    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
+}
+
+w4a8_status w4a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                          const uint8_t *Wp, int ldp, const float *sw, int N, const float *bias,
+                          unsigned flags, void *Y, int ldy, void *stream) {
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldq < K || ldq % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
+    return run_product(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+                       static_cast<cudaStream_t>(stream));
+}
+
+unsigned w4a8_last_path(void) { return t_last_path; }
+
+w4a8_status w4a8_get_device_status(int clear, void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return W4A8_ERR_CUDA;
+    }
+    return v;
+}
+
+const char *w4a8_status_string(w4a8_status s) {
+    switch (s) {
+        case W4A8_OK: return "ok";
+        case W4A8_ERR_INVALID_ARG: return "invalid argument";
+        case W4A8_ERR_UNSUPPORTED: return "unsupported device or shape";
+        case W4A8_ERR_WORKSPACE: return "workspace missing or too small";
+        case W4A8_ERR_CUDA: return "CUDA error";
+        case W4A8_ERR_TIMEOUT: return "bounded wait in a kernel ran out";
+        case W4A8_ERR_BOUNDS: return "out-of-range index caught in a kernel";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

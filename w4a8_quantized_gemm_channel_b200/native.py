@@ -1,0 +1,182 @@
+"""Thin ctypes binding over libw4a8.so (the C ABI declared in include/w4a8.h).
+
+Argument marshalling only: torch tensors -> device pointers, strides and the
+current CUDA stream. Every step of the layer runs in the library's kernels;
+torch only allocates device memory. If the library is missing this module
+raises at import time: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a8.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(7)
+
+RELU = 0x01
+OUT_F32, OUT_BF16, OUT_S32 = 0x00, 0x02, 0x04
+PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TC = 0x00, 0x10, 0x20, 0x30
+MAX_K = 2097152
+
+_OUT = {"f32": OUT_F32, "bf16": OUT_BF16, "s32": OUT_S32}
+_OUT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "s32": torch.int32}
+_PATH = {"auto": PATH_AUTO, "generic": PATH_GENERIC, "decode": PATH_DECODE, "tc": PATH_TC}
+PATH_NAMES = {v: k for k, v in _PATH.items()}
+
+# Every symbol include/w4a8.h declares, with its ctypes signature.
+_P, _I, _U, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
+SIGNATURES = {
+    "w4a8_packed_ld": (_I, [_I]),
+    "w4a8_act_ld": (_I, [_I]),
+    "w4a8_workspace_size": (_S, [_I, _I]),
+    "w4_quantize_pack": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
+    "a8_quantize_rows": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
+    "w4a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
+    "w4a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
+    "w4a8_last_path": (_U, []),
+    "w4a8_get_device_status": (_I, [_I, _P]),
+    "w4a8_status_string": (ctypes.c_char_p, [_I]),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libw4a8.so not found at {LIB_PATH}; build it with "
+            "`python -m w4a8_quantized_gemm_channel_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class W4A8Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib.w4a8_status_string(status).decode()} (status {status})")
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise W4A8Error(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _rowmajor(t: torch.Tensor, name: str):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def packed_ld(k: int) -> int:
+    return lib.w4a8_packed_ld(k)
+
+
+def act_ld(k: int) -> int:
+    return lib.w4a8_act_ld(k)
+
+
+def workspace_size(m: int, k: int) -> int:
+    return lib.w4a8_workspace_size(m, k)
+
+
+def flags_for(relu: bool = False, out: str = "f32", path: str = "auto") -> int:
+    return (RELU if relu else 0) | _OUT[out] | _PATH[path]
+
+
+def w4_quantize_pack(w: torch.Tensor, wp: torch.Tensor | None = None,
+                     sw: torch.Tensor | None = None, stream=None):
+    """W[K][N] float32 (CUDA) -> (Wp[N][ldp] uint8, sw[N] float32)."""
+    ldw = _rowmajor(w, "W")
+    k, n = w.shape
+    if wp is None:
+        wp = torch.empty((n, packed_ld(k)), dtype=torch.uint8, device=w.device)
+    if sw is None:
+        sw = torch.empty(n, dtype=torch.float32, device=w.device)
+    ldp = _rowmajor(wp, "Wp")
+    _check(lib.w4_quantize_pack(_ptr(w), k, n, ldw, _ptr(wp), ldp, _ptr(sw), _stream(stream)),
+           "w4_quantize_pack")
+    return wp, sw
+
+
+def a8_quantize_rows(x: torch.Tensor, xq: torch.Tensor | None = None,
+                     sx: torch.Tensor | None = None, stream=None):
+    """X[M][K] float32 (CUDA) -> (Xq[M][ldq] int8, sx[M] float32)."""
+    ldx = _rowmajor(x, "X")
+    m, k = x.shape
+    if xq is None:
+        xq = torch.empty((m, act_ld(k)), dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty(m, dtype=torch.float32, device=x.device)
+    ldq = _rowmajor(xq, "Xq")
+    _check(lib.a8_quantize_rows(_ptr(x), m, k, ldx, _ptr(xq), ldq, _ptr(sx), _stream(stream)),
+           "a8_quantize_rows")
+    return xq, sx
+
+
+def _out_tensor(y, m, n, out, device):
+    if y is None:
+        y = torch.empty((m, n), dtype=_OUT_DTYPE[out], device=device)
+    return y, _rowmajor(y, "Y")
+
+
+def w4a8_linear(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
+                bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
+                path: str = "auto", y: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[M][N] = dequant(quant8(X) @ unpack(Wp)^T) (+bias, ReLU) for X[M][K] float32."""
+    ldx = _rowmajor(x, "X")
+    ldp = _rowmajor(wp, "Wp")
+    m, k = x.shape
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, x.device)
+    need = workspace_size(m, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(lib.w4a8_linear(_ptr(x), m, k, ldx, _ptr(wp), ldp, _ptr(sw), n, _ptr(bias),
+                           flags_for(relu, out, path), _ptr(y), ldy, _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream)),
+           "w4a8_linear")
+    return y
+
+
+def w4a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor,
+                  sw: torch.Tensor, bias: torch.Tensor | None = None, relu: bool = False,
+                  out: str = "f32", path: str = "auto", y: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Y from INT8 activations Xq[M][ldq] (first k bytes of each row) and sx[M]."""
+    ldq = _rowmajor(xq, "Xq")
+    ldp = _rowmajor(wp, "Wp")
+    m = xq.shape[0]
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, xq.device)
+    _check(lib.w4a8_linear_q(_ptr(xq), m, k, ldq, _ptr(sx), _ptr(wp), ldp, _ptr(sw), n,
+                             _ptr(bias), flags_for(relu, out, path), _ptr(y), ldy,
+                             _stream(stream)),
+           "w4a8_linear_q")
+    return y
+
+
+def last_path() -> str:
+    return PATH_NAMES.get(lib.w4a8_last_path(), "none")
+
+
+def get_device_status(clear: bool = False, stream=None) -> int:
+    return lib.w4a8_get_device_status(int(clear), _stream(stream))
