@@ -165,6 +165,15 @@ class DecodeWorkload:
 
 # ------------------------------------------------------------ timing core ---
 
+def max_over_ranks(torch, dist, value: float, device) -> float:
+    """The slowest rank's time (every rank gets it); identity on one rank."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def build_graphs(torch, wl, nsteps):
     """CUDA graphs of GRAPH_STEPS steps (and one for the remainder)."""
     graphs = []
@@ -323,7 +332,7 @@ def oracle_decode_rate(budget_s: float, min_steps: int = 1):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    budget = min(120.0, max(10.0, 0.01 * (args.steps + args.warmup)))
+    budget = args.cpu_budget
     gbs, t, chunks, cols = oracle_decode_rate(budget)
     sample = (f"{chunks} samples of {cols} output channels x full K=4096 at M=1,4,16 "
               f"({t:.1f} s single-threaded)")
@@ -391,10 +400,7 @@ def main():
     time.sleep(0.3)
     ms = time_steps(torch, wl, args.steps, args.warmup, dist)
     ck = clocks.stop()
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(torch, dist, ms, device)
     bytes_step = wl.bytes_per_step()
     value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9
 

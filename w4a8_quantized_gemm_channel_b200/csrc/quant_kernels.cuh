@@ -12,39 +12,57 @@
 namespace w4a8 {
 
 // ---------------------------------------------------------------------------
-// Weight pass 1: column abs-max. W is [K][ldw] (columns = output channels), so
-// a warp reads 32 consecutive columns of one row (128 contiguous bytes) and
-// the block's 8 warps walk disjoint rows of a K-slice. The per-column maxima
-// of all K-slices meet in amax_bits[n] through an integer atomicMax on the
-// float bit patterns (valid because every value is >= +0).
-// grid = (ceil(N/32), k_splits), block = (32, 8).
+// Weight pass 1: column abs-max. W is [K][ldw] (columns = output channels).
+// VEC = 4: a warp reads 128 consecutive columns of one row as float4 (512
+// contiguous bytes); VEC = 1 is the scalar form for unaligned layouts. The
+// block's 8 warps walk disjoint rows of a K-slice, 4 rows in flight each;
+// the per-column maxima of all K-slices meet in amax_bits[n] through an
+// integer atomicMax on the float bit patterns (valid: every value >= +0).
+// grid = (ceil(N / (32 * VEC)), k_splits), block = 256.
 // ---------------------------------------------------------------------------
+template <int VEC>
 __global__ void __launch_bounds__(256)
 k_col_absmax(const float *__restrict__ W, int K, int N, int ldw, int rows_per_split,
              unsigned *__restrict__ amax_bits) {
-    __shared__ float red[8][33];
-    const int n = blockIdx.x * 32 + threadIdx.x;
+    __shared__ float red[8][32 * VEC + 1];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = (blockIdx.x * 32 + lane) * VEC;
     const int k0 = blockIdx.y * rows_per_split;
     const int k1 = min(K, k0 + rows_per_split);
-    float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
+    float m[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) m[c] = 0.0f;
+    auto take = [&](const float *p) {
+        if constexpr (VEC == 4) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+            m[0] = fmaxf(m[0], fabsf(v.x)); m[1] = fmaxf(m[1], fabsf(v.y));
+            m[2] = fmaxf(m[2], fabsf(v.z)); m[3] = fmaxf(m[3], fabsf(v.w));
+        } else {
+            m[0] = fmaxf(m[0], fabsf(__ldg(p)));
+        }
+    };
     if (n < N) {
         const float *col = W + n;
-        int k = k0 + threadIdx.y;
+        int k = k0 + warp;
         for (; k + 24 < k1; k += 32) {
-            m0 = fmaxf(m0, fabsf(__ldg(col + (size_t)k * ldw)));
-            m1 = fmaxf(m1, fabsf(__ldg(col + (size_t)(k + 8) * ldw)));
-            m2 = fmaxf(m2, fabsf(__ldg(col + (size_t)(k + 16) * ldw)));
-            m3 = fmaxf(m3, fabsf(__ldg(col + (size_t)(k + 24) * ldw)));
+            take(col + (size_t)k * ldw);
+            take(col + (size_t)(k + 8) * ldw);
+            take(col + (size_t)(k + 16) * ldw);
+            take(col + (size_t)(k + 24) * ldw);
         }
-        for (; k < k1; k += 8) m0 = fmaxf(m0, fabsf(__ldg(col + (size_t)k * ldw)));
+        for (; k < k1; k += 8) take(col + (size_t)k * ldw);
     }
-    red[threadIdx.y][threadIdx.x] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-    __syncthreads();
-    if (threadIdx.y == 0 && n < N) {
-        float m = red[0][threadIdx.x];
 #pragma unroll
-        for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i][threadIdx.x]);
-        atomicMax(&amax_bits[n], __float_as_uint(m));
+    for (int c = 0; c < VEC; ++c) red[warp][lane * VEC + c] = m[c];
+    __syncthreads();
+    for (int c = threadIdx.x; c < 32 * VEC; c += 256) {
+        const int nn = blockIdx.x * 32 * VEC + c;
+        if (nn < N) {
+            float a = red[0][c];
+#pragma unroll
+            for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i][c]);
+            atomicMax(&amax_bits[nn], __float_as_uint(a));
+        }
     }
 }
 
@@ -53,55 +71,71 @@ __device__ __forceinline__ float weight_scale_from_amax(unsigned bits) {
     return a == 0.0f ? 1.0f : __fdiv_rn(7.0f, a);
 }
 
+// Four codes (one per byte of w, each in [-8, 7]) -> 16 bits of nibbles,
+// the code of byte 0 in the lowest nibble.
+__device__ __forceinline__ uint32_t pack4_nibbles(uint32_t w) {
+    uint32_t x = w & 0x0F0F0F0Fu;
+    uint32_t y = (x | (x >> 4)) & 0x00FF00FFu;
+    return (y | (y >> 8)) & 0xFFFFu;
+}
+
 // ---------------------------------------------------------------------------
-// Weight pass 2: quantize and pack a tile of 64 k x 32 output channels.
-// Reads are row-coalesced (a warp reads 32 columns of one row); the codes are
+// Weight pass 2: quantize and pack a tile of 64 k x (32 * VEC) output
+// channels. Reads are row-coalesced (float4 per lane for VEC = 4); codes are
 // transposed through shared memory so each output channel's 32 bytes of
-// packed nibbles leave as two 16-byte stores. Tiles cover k in [0, 2*ldp), so
-// every byte of every packed row (pad bytes included) is written.
-// grid = (ceil(N/32), ceil(2*ldp/64)), block = (32, 8).
+// packed nibbles leave as two 16-byte stores. Tiles cover k in [0, 2*ldp),
+// so every byte of every packed row (pad bytes included) is written.
+// grid = (ceil(N / (32 * VEC)), ceil(2*ldp / 64)), block = 256.
 // ---------------------------------------------------------------------------
+template <int VEC>
 __global__ void __launch_bounds__(256)
 k_quant_pack(const float *__restrict__ W, int K, int N, int ldw,
              const unsigned *__restrict__ amax_bits, uint8_t *__restrict__ Wp, int ldp) {
-    __shared__ int8_t qs[32][64 + 4];
-    const int n = blockIdx.x * 32 + threadIdx.x;
+    constexpr int COLS = 32 * VEC;
+    constexpr int QS = 64 + 16;  // row pitch of the transposed codes (16-byte aligned)
+    __shared__ __align__(16) int8_t qs[COLS][QS];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nb = blockIdx.x * COLS;
+    const int n = nb + lane * VEC;
     const int k0 = blockIdx.y * 64;
-    float s = 1.0f;
-    if (n < N) s = weight_scale_from_amax(__ldg(amax_bits + n));
+    float s[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) s[c] = (n + c < N) ? weight_scale_from_amax(__ldg(amax_bits + n + c)) : 1.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int kk = threadIdx.y + 8 * i;
+        const int kk = warp + 8 * i;
         const int k = k0 + kk;
-        int q = 0;
-        if (n < N && k < K) {
-            float t = __fmul_rn(__ldg(W + (size_t)k * ldw + n), s);
-            q = clampi(__float2int_rn(t), -8, 7);
+        float v[VEC];
+        if (k < K && n < N) {
+            if constexpr (VEC == 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(W + (size_t)k * ldw + n));
+                v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+            } else {
+                v[0] = __ldg(W + (size_t)k * ldw + n);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) v[c] = 0.0f;
         }
-        qs[threadIdx.x][kk] = (int8_t)q;
+#pragma unroll
+        for (int c = 0; c < VEC; ++c)
+            qs[lane * VEC + c][kk] = (int8_t)clampi(__float2int_rn(__fmul_rn(v[c], s[c])), -8, 7);
     }
     __syncthreads();
-    const int t = threadIdx.y * 32 + threadIdx.x;
-    if (t < 64) {
-        const int r = t >> 1, h = t & 1;
-        const int nn = blockIdx.x * 32 + r;
+    // 2 threads per output channel row, 16 packed bytes (32 codes) each.
+    for (int tt = threadIdx.x; tt < 2 * COLS; tt += 256) {
+        const int r = tt >> 1, h = tt & 1;
+        const int nn = nb + r;
         const int byte0 = k0 / 2 + 16 * h;  // a multiple of 16, as is ldp
         if (nn < N && byte0 < ldp) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t v = 0;
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int kk = 32 * h + 8 * j + 2 * b;
-                    uint32_t lo = (uint32_t)(uint8_t)qs[r][kk] & 0xFu;
-                    uint32_t hi = (uint32_t)(uint8_t)qs[r][kk + 1] & 0xFu;
-                    v |= (lo | (hi << 4)) << (8 * b);
-                }
-                w[j] = v;
-            }
-            *reinterpret_cast<uint4 *>(Wp + (size_t)nn * ldp + byte0) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            const uint4 a = *reinterpret_cast<const uint4 *>(&qs[r][32 * h]);
+            const uint4 b = *reinterpret_cast<const uint4 *>(&qs[r][32 * h + 16]);
+            uint4 o;
+            o.x = pack4_nibbles(a.x) | (pack4_nibbles(a.y) << 16);
+            o.y = pack4_nibbles(a.z) | (pack4_nibbles(a.w) << 16);
+            o.z = pack4_nibbles(b.x) | (pack4_nibbles(b.y) << 16);
+            o.w = pack4_nibbles(b.z) | (pack4_nibbles(b.w) << 16);
+            *reinterpret_cast<uint4 *>(Wp + (size_t)nn * ldp + byte0) = o;
         }
     }
 }

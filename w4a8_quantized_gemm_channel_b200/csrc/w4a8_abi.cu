@@ -181,18 +181,28 @@ w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp,
     unsigned *amax = reinterpret_cast<unsigned *>(sw);
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * (size_t)N, s);
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
-    // K-slices so that the abs-max pass puts a few blocks on every SM.
-    const int col_blocks = (N + 31) / 32;
-    int splits = (4 * dev.sm_count + col_blocks - 1) / col_blocks;
+    // VEC = 4 (float4 rows) when the layout allows it.
+    const bool v4 = (N % 4 == 0) && (ldw % 4 == 0) && aligned16(W);
+    const int cols = v4 ? 128 : 32;
+    const int col_blocks = (N + cols - 1) / cols;
+    // K-slices so that the abs-max pass puts several blocks on every SM.
+    int splits = (6 * dev.sm_count + col_blocks - 1) / col_blocks;
     splits = splits < 1 ? 1 : splits;
     int rows = (K + splits - 1) / splits;
-    rows = round_up(rows < 64 ? 64 : rows, 8);
+    rows = round_up(rows < 64 ? 64 : rows, 32);
     splits = (K + rows - 1) / rows;
-    k_col_absmax<<<dim3(col_blocks, splits), dim3(32, 8), 0, s>>>(W, K, N, ldw, rows, amax);
+    if (splits > 65535) return W4A8_ERR_UNSUPPORTED;
+    if (v4)
+        k_col_absmax<4><<<dim3(col_blocks, splits), 256, 0, s>>>(W, K, N, ldw, rows, amax);
+    else
+        k_col_absmax<1><<<dim3(col_blocks, splits), 256, 0, s>>>(W, K, N, ldw, rows, amax);
     if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
     const int kblocks = (2 * ldp + 63) / 64;
     if (kblocks > 65535) return W4A8_ERR_UNSUPPORTED;
-    k_quant_pack<<<dim3(col_blocks, kblocks), dim3(32, 8), 0, s>>>(W, K, N, ldw, amax, Wp, ldp);
+    if (v4)
+        k_quant_pack<4><<<dim3(col_blocks, kblocks), 256, 0, s>>>(W, K, N, ldw, amax, Wp, ldp);
+    else
+        k_quant_pack<1><<<dim3(col_blocks, kblocks), 256, 0, s>>>(W, K, N, ldw, amax, Wp, ldp);
     if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
     k_weight_scale_finalize<<<(N + 255) / 256, 256, 0, s>>>(sw, N);
     return from_cuda(cudaGetLastError());
