@@ -163,6 +163,58 @@ class DecodeWorkload:
                 "activations": "N(0,1), 8 input channels x20"}
 
 
+class PrefillWorkload:
+    """M = 2048, K = 4096, N = 11008 (MLP up-projection shape); weights
+    N(0, 0.02); X N(0, 1) with 0.5% of input channels x20. One step = one
+    w4a8_linear (activation quantization + tensor-core GEMM + epilogue)."""
+    name = "prefill"
+
+    def __init__(self, torch, native, synth, device, l2_bytes, relu=False):
+        self.torch, self.nat = torch, native
+        c = synth.prefill_case()
+        self.M, self.K, self.N = c.x.shape[0], c.w.shape[0], c.w.shape[1]
+        self.MS = (self.M,)
+        self.relu = relu
+        wd = torch.from_numpy(c.w).to(device)
+        self.wd = wd
+        wp, sw = native.w4_quantize_pack(wd)
+        per_set = wp.numel() + 4 * self.M * self.K + 4 * self.M * self.N
+        self.pool = max(2, -(-3 * l2_bytes // per_set))
+        self.wp = [wp.clone() for _ in range(self.pool)]
+        self.sw = [sw.clone() for _ in range(self.pool)]
+        self.x_host = {self.M: c.x}
+        x = torch.from_numpy(c.x).to(device)
+        self.xs = [x.clone() for _ in range(self.pool)]
+        self.x = {self.M: x}
+        self.ys = [torch.empty((self.M, self.N), dtype=torch.float32, device=device) for _ in range(self.pool)]
+        self.y = {self.M: self.ys[0]}
+        self.ws = {self.M: torch.empty(native.workspace_size(self.M, self.K), dtype=torch.uint8, device=device)}
+        self.slot = 0
+        self.pool_bytes = self.pool * per_set
+
+    def bytes_per_step(self):
+        return self.N * self.nat.packed_ld(self.K) + 4 * self.N + 4 * self.M * self.K + 4 * self.M * self.N
+
+    def ops_per_step(self):
+        return 2 * self.M * self.N * self.K
+
+    def launches_per_step(self):
+        return 2
+
+    def step(self):
+        s = self.slot
+        self.slot = (self.slot + 1) % self.pool
+        self.nat.w4a8_linear(self.xs[s], self.wp[s], self.sw[s], relu=self.relu, y=self.ys[s],
+                             workspace=self.ws[self.M])
+
+    def config(self):
+        return {"workload": f"prefill single linear M={self.M} K={self.K} N={self.N}"
+                            + (" +ReLU" if self.relu else ""),
+                "M": self.M, "K": self.K, "N": self.N,
+                "l2": f"inputs larger than L2: {self.pool} distinct X/W/Y sets "
+                      f"({self.pool_bytes / 1e6:.0f} MB) rotate across launches"}
+
+
 # ------------------------------------------------------------ timing core ---
 
 def max_over_ranks(torch, dist, value: float, device) -> float:
@@ -260,6 +312,35 @@ def time_kernel_only(torch, nat, wl):
     return out
 
 
+def time_gemm_only(torch, nat, wl, reps=20):
+    """Average device time per tensor-core GEMM launch (w4a8_linear_q on INT8
+    activations) over the rotating buffer sets."""
+    m = wl.M
+    xqs = [nat.a8_quantize_rows(x) for x in wl.xs]
+    def run():
+        for i in range(wl.pool):
+            xq, sx = xqs[i]
+            nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        g.replay()
+    stop.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(stop) / (reps * wl.pool)
+
+
 def time_quantize_pack(torch, nat, wl):
     """The offline weight pass (steps 1-2) on the decode weight matrix."""
     wp, sw = nat.w4_quantize_pack(wl.wd)
@@ -349,6 +430,85 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False):
+    wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu)
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_steps(torch, wl, args.steps, args.warmup, dist)
+    ck = clocks.stop()
+    ms = max_over_ranks(torch, dist, ms, device)
+    tops = world * args.steps * wl.ops_per_step() / (ms * 1e-3) / 1e12
+    g_ms = time_gemm_only(torch, native, wl)
+    peaks, kind = measured_peaks()
+    peak = INT8_OVER_BF16 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    achieved = wl.ops_per_step() / (g_ms * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": round(tops, 2), "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8xs4->s32",
+            "data": "synthetic", "config": wl.config(),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                         "unit": "TOPS", "frac": round(achieved / peak, 4),
+                         "peak_source": f"{kind} bf16_tflops x {INT8_OVER_BF16:g} (nominal int8/bf16)",
+                         "traffic": None, "kernel": "k_gemm_tc (w4a8_linear_q, rotating buffers)",
+                         "us": round(g_ms * 1e3, 2)},
+            "gpu_launches": args.steps * wl.launches_per_step(), "clocks": ck}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_sweep(torch, native, synth, device, props):
+    """Kernel time per shape of the Gemma3-1B stack and the 70B-shaped layers
+    (w4a8_linear end to end on device-resident inputs, back-to-back in a
+    graph over rotating weight copies)."""
+    peaks, _ = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    tc = INT8_OVER_BF16 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    shapes = [("gemma_" + nm, k, n, m, 0.02) for (nm, k, n) in synth.GEMMA_PROJ for m in synth.GEMMA_MS]
+    shapes += [(f"llama70_{k}x{n}", k, n, m, 0.01) for (k, n) in synth.LLAMA70_SHAPES for m in synth.LLAMA70_MS]
+    for name, k, n, m, std in shapes:
+        w = torch.from_numpy(synth.linear_weights(k, n, std, seed=3)).to(device)
+        wp, sw = native.w4_quantize_pack(w)
+        del w
+        x = torch.from_numpy(synth.linear_activations(m, k, seed=3)[0]).to(device)
+        per = wp.numel() + 4 * m * k + 4 * m * n
+        pool = max(2, min(64, -(-3 * props.L2_cache_size // per)))
+        wps = [wp.clone() for _ in range(pool)]
+        sws = [sw.clone() for _ in range(pool)]
+        y = torch.empty((m, n), dtype=torch.float32, device=device)
+        ws = torch.empty(native.workspace_size(m, k), dtype=torch.uint8, device=device)
+
+        def run():
+            for i in range(pool):
+                native.w4a8_linear(x, wps[i], sws[i], y=y, workspace=ws)
+        run()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(3, int(2e9 // max(1, 2 * m * n * k * pool)))
+        reps = min(reps, 200)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(reps):
+            g.replay()
+        stop.record()
+        torch.cuda.synchronize()
+        us = start.elapsed_time(stop) * 1e3 / (reps * pool)
+        nbytes = n * native.packed_ld(k) + 4 * n + 4 * m * k + 4 * m * n
+        ops = 2 * m * n * k
+        gbs = nbytes / (us * 1e-6) / 1e9
+        tops = ops / (us * 1e-6) / 1e12
+        frac = max(gbs / hbm, tops / tc)
+        print(json.dumps({"shape": name, "M": m, "K": k, "N": n, "us": round(us, 3),
+                          "GBs": round(gbs, 1), "TOPS": round(tops, 2), "roofline_frac": round(frac, 4),
+                          "path": native.last_path()}), flush=True)
+        del wps, sws, wp, sw, x, y, ws, g
+        torch.cuda.empty_cache()
+
+
 # --------------------------------------------------------------- main ---
 
 def main():
@@ -359,6 +519,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU work for the oracle baseline")
+    ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep"],
+                    default="decode",
+                    help="decode (the headline line), prefill (M=2048 K=4096 N=11008), "
+                         "or a per-shape sweep of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -393,6 +557,13 @@ def main():
 
     from w4a8_quantized_gemm_channel_b200 import native, synth
     props = torch.cuda.get_device_properties(device)
+    if args.workload in ("prefill", "prefill-relu"):
+        run_prefill(args, torch, native, synth, device, props, dist, world, rank,
+                    relu=args.workload == "prefill-relu")
+        return
+    if args.workload == "sweep":
+        run_sweep(torch, native, synth, device, props)
+        return
     wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size)
 
     clocks = ClockSampler(local)

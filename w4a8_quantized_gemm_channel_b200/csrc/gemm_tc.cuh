@@ -39,7 +39,13 @@ constexpr int MMA_K = 32;          // k per kind::i8 instruction
 // 6 stages: 144 KB of shared memory, which also keeps a second CTA (that
 // would block in tcgen05.alloc of the whole TMEM) off the SM.
 constexpr int STAGES = 6;
-constexpr int NUM_THREADS = 384;
+// Unpack warpgroups: stage s is unpacked by warpgroup s % UNPACK_WG, so the
+// groups overlap their shared-memory reads, integer work and TMEM stores.
+constexpr int UNPACK_WG = 3;
+static_assert(STAGES % UNPACK_WG == 0, "each warpgroup owns fixed ring slots");
+constexpr int FIRST_UNPACK_WARP = 4;
+constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + 4 * UNPACK_WG;
+constexpr int NUM_THREADS = 32 * (FIRST_EPI_WARP + 4);
 constexpr int TMEM_COLS = 512;
 constexpr int A_COLS = BK / 4;     // TMEM columns per A slot (4 INT8 per column)
 constexpr int W_TILE_BYTES = BM * BK / 2;
@@ -54,6 +60,7 @@ struct alignas(1024) Smem {
     uint64_t acc_full[2];                // accumulator ready for the epilogue
     uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
     uint64_t mma_done;                   // final drain of the MMA pipe
+    float rsx[BT];                       // 1/sx of the epilogue's current token tile
     uint32_t tmem_base;
     int abort;
 };
@@ -173,20 +180,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 ptx::mbar_wait_drain(&sm.mma_done, 0);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= FIRST_UNPACK_WARP && warp < FIRST_EPI_WARP) {
         // ---------------------------------------------------- weight unpack
         // Thread r owns output-channel row r of the tile: 64 packed bytes per
         // stage, read from the 64B-swizzled tile (16-byte chunk c of row r
         // sits at chunk c ^ ((r >> 1) & 3)), expanded to 128 INT8 in k order
-        // and stored to TMEM lane r, 32 columns.
+        // and stored to TMEM lane r, 32 columns. Warpgroup wg takes the
+        // pipeline iterations it with it % UNPACK_WG == wg.
         const int q = warp & 3;
+        const int wg = (warp - FIRST_UNPACK_WARP) >> 2;
         const int r = q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
+        int it = 0;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            for (int kb = 0; kb < num_kb; ++kb) {
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                if (it % UNPACK_WG != wg) {
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    continue;
+                }
                 // every lane waits (each then sees the TMA data); the outcome is
                 // made warp-uniform before the warp-collective tcgen05.st
                 ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sm.full[stage], phase, abort));
@@ -214,9 +228,20 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= FIRST_EPI_WARP) {
         // ---------------------------------------------------- epilogue
+        // Thread owns output channel n (TMEM lane); per tile it first fills a
+        // table of 1/sx for the tile's tokens (one entry per thread), then
+        // dequantizes 32 tokens per tcgen05.ld.
+        //
+        // y = acc / (sx * sw) without a per-element division: with
+        // r = (1/sx) * (1/sw), an approximation of 1/d for d = sx * sw, take
+        // q0 = f * r and correct it once with the exact remainder,
+        // q = q0 + (f - q0 * d) * r (two FMAs; Markstein's quotient
+        // correction). The result is the correctly rounded quotient in
+        // practice and always within a few ulp (<< 1e-6 relative).
         const int q = warp & 3;
+        const int et = threadIdx.x - 32 * FIRST_EPI_WARP;  // 0..127
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         int buf = 0;
         uint32_t acc_phase = 0;
@@ -224,13 +249,23 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
         const bool relu = (flags & W4A8_RELU) != 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int n_tile = tile / tiles_m, m_tile = tile % tiles_m;
-            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sm.acc_full[buf], acc_phase, abort))) break;
+            const int m_base = m_tile * BT;
+            // reciprocal scales of this tile's tokens (the previous tile's
+            // readers are past the named barrier at its end)
+            for (int c = et; c < BT; c += 128) {
+                const int m = m_base + c;
+                sm.rsx[c] = m < M ? __frcp_rn(__ldg(sx + m)) : 0.0f;
+            }
+            // One decision for all four epilogue warps (this barrier also
+            // publishes rsx): a warp that gave up must not leave the others
+            // waiting at a named barrier.
+            if (!ptx::bar_and(1, 128, ptx::mbar_wait(&sm.acc_full[buf], acc_phase, abort))) break;
             ptx::tc_fence_after();
             const int n = n_tile * BM + q * 32 + lane;
             const bool n_ok = n < N;
             const float swn = n_ok ? __ldg(sw + n) : 1.0f;
+            const float rswn = __frcp_rn(swn);
             const float bn = (bias && n_ok) ? __ldg(bias + n) : 0.0f;
-            const int m_base = m_tile * BT;
 #pragma unroll 1
             for (int c0 = 0; c0 < BT; c0 += 32) {
                 uint32_t v[32];
@@ -247,7 +282,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                         if (fmt == W4A8_OUT_S32) {
                             static_cast<int32_t *>(Y)[off] = acc;
                         } else {
-                            float y = __fdiv_rn(__int2float_rn(acc), __fmul_rn(__ldg(sx + m), swn));
+                            const float f = __int2float_rn(acc);
+                            const float d = __fmul_rn(__ldg(sx + m), swn);
+                            const float r = __fmul_rn(sm.rsx[c0 + j], rswn);
+                            const float q0 = __fmul_rn(f, r);
+                            const float e = __fmaf_rn(-q0, d, f);
+                            float y = __fmaf_rn(e, r, q0);
                             if (bias) y = __fadd_rn(y, bn);
                             if (relu) y = y > 0.0f ? y : 0.0f;
                             if (fmt == W4A8_OUT_BF16)
@@ -262,6 +302,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&sm.acc_empty[buf]);
             if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+            ptx::bar_sync(1, 128);  // rsx is rewritten next tile
         }
     }
 
