@@ -149,6 +149,34 @@ W4A8_API w4a8_status w4a8_linear_q(const int8_t *Xq, int M, int K, int ldq, cons
                           const float *bias, unsigned flags,
                           void *Y, int ldy, void *stream);
 
+/*
+ * w4a8_linear_noalloc - w4a8_linear for callers that cannot allocate device
+ * memory: a host that hands this library only its input and output buffers
+ * (a plugin or custom-op interface with no allocator of its own), or code
+ * that must not call cudaMalloc because it can block or synchronize work
+ * that is already running. It performs the same computation as w4a8_linear
+ * (steps 3-6), but keeps the INT8 activations and their scales in scratch
+ * memory the library owns: one static device array of
+ * W4A8_NOALLOC_SCRATCH_BYTES bytes per GPU, which every GPU that loads the
+ * library holds until the process exits. The pages (Keras INT4 guide) have
+ * no counterpart of this entry point; it is an addition for such callers.
+ *   Arguments as for w4a8_linear, without the workspace.
+ *   Returns W4A8_ERR_WORKSPACE when w4a8_workspace_size(M, K) exceeds
+ *   W4A8_NOALLOC_SCRATCH_BYTES (nothing is enqueued then).
+ *   The first call on each device looks up the array's device address with
+ *   that device current (the set-up is done once per device); make that first
+ *   call before any stream capture on the device.
+ *   Every call shares the one array: calls whose work can overlap on the GPU
+ *   (different streams, or different host threads) race on it and corrupt
+ *   each other's results; order them on one stream. Each call rewrites every
+ *   byte it reads, so nothing left by an earlier call leaks into the result.
+ */
+#define W4A8_NOALLOC_SCRATCH_BYTES (16u << 20)
+W4A8_API w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx,
+                                         const uint8_t *Wp, int ldp, const float *sw, int N,
+                                         const float *bias, unsigned flags,
+                                         void *Y, int ldy, void *stream);
+
 /* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
  * last successful w4a8_linear / w4a8_linear_q call enqueued; 0 if none. */
 W4A8_API unsigned w4a8_last_path(void);

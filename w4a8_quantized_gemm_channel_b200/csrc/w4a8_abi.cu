@@ -154,6 +154,27 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     return W4A8_OK;
 }
 
+// Scratch of w4a8_linear_noalloc: a file-scope device array, so callers that
+// cannot allocate still get somewhere to keep the INT8 activations.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_BYTES];
+
+// The array's device address, looked up once per device with that device
+// current. In host code the symbol g_noalloc_scratch is only a host-side
+// stand-in and must never be handed to a kernel.
+void *noalloc_scratch_ptr() {
+    static std::mutex mu;
+    static void *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
+
 }  // namespace
 }  // namespace w4a8
 
@@ -258,6 +279,25 @@ w4a8_status w4a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *
     if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
     return run_product(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
                        static_cast<cudaStream_t>(stream));
+}
+
+w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp,
+                                const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                                void *stream) {
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
+    if (w4a8_workspace_size(M, K) > (size_t)W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    void *scratch = noalloc_scratch_ptr();
+    if (!scratch) return W4A8_ERR_CUDA;
+    const Workspace ws = carve_workspace(scratch, M, K);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
+    if (st != W4A8_OK) return st;
+    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
 }
 
 unsigned w4a8_last_path(void) { return t_last_path; }

@@ -37,6 +37,7 @@ SIGNATURES = {
     "a8_quantize_rows": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     "w4a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
     "w4a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
+    "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_last_path": (_U, []),
     "w4a8_get_device_status": (_I, [_I, _P]),
     "w4a8_status_string": (ctypes.c_char_p, [_I]),
@@ -171,6 +172,26 @@ def w4a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor,
                              _ptr(bias), flags_for(relu, out, path), _ptr(y), ldy,
                              _stream(stream)),
            "w4a8_linear_q")
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def w4a8_linear_noalloc(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
+                        bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
+                        path: str = "auto", y: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """w4a8_linear without a caller workspace: the INT8 activations live in the
+    library's fixed per-device scratch array (see include/w4a8.h)."""
+    ldx = _rowmajor(x, "X")
+    ldp = _rowmajor(wp, "Wp")
+    m, k = x.shape
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, x.device)
+    _check(lib.w4a8_linear_noalloc(_ptr(x), m, k, ldx, _ptr(wp), ldp, _ptr(sw), n, _ptr(bias),
+                                   flags_for(relu, out, path), _ptr(y), ldy, _stream(stream)),
+           "w4a8_linear_noalloc")
     return y
 
 
