@@ -292,3 +292,53 @@ def test_llama70_shapes_sampled(nat, shape):
         c = synth.llama70_case(shape, m)
         rows = np.unique(np.concatenate([[0, m - 1], rng.integers(0, m, size=4)]))
         _sampled_check(nat, c.x, None, wpd, swd, rows, cols)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_linear_q_full_code_range(nat, path):
+    """Every INT4 code, -8 included (the packed format allows it even though
+    abs-max quantization never produces it), against every INT8 value."""
+    rng = synth.rng_for(12, 0)
+    m, k, n = 40, 768, 136
+    q = rng.integers(-8, 8, size=(n, k)).astype(np.int8)
+    q[:, :16] = -8
+    xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+    xq[:, :16] = -127
+    sx = (rng.random(m) + 0.5).astype(np.float32)
+    sw = (rng.random(n) + 0.5).astype(np.float32)
+    wp = oracle.w4_pack(q)
+    acc = nat.w4a8_linear_q(dev(xq), dev(sx), k, dev(wp), dev(sw), out="s32", path=path)
+    assert np.array_equal(host(acc), oracle.gemm_s32(xq, k, wp))
+    y = nat.w4a8_linear_q(dev(xq), dev(sx), k, dev(wp), dev(sw), path=path)
+    assert_f32_close(host(y), oracle.linear_q(xq, sx, wp, sw, k))
+
+
+def test_tc_large_k_uses_sign_extension(nat):
+    """K above the limit of the tensor-core kernel's 16*q byte trick
+    (16 * 128 * 127 * K must stay below 2^31) still gives exact results."""
+    m, k, n = 20, 140000, 16
+    x, w, _ = _case(m, k, n, seed=900)
+    wp, sw = oracle.w4_quantize_pack(w)
+    acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32", path="tc")
+    assert np.array_equal(host(acc), oracle.linear(x, wp, sw, k, out="s32"))
+
+
+@pytest.mark.parametrize("m,k,n,pad", [(1, 4096, 64, 0), (5, 1001, 40, 3), (8, 2048, 33, 0)])
+def test_decode_linear_matches_quantize_then_linear_q(nat, m, k, n, pad):
+    """w4a8_linear on the decode path must agree bit for bit with quantizing
+    first (a8_quantize_rows) and multiplying after (w4a8_linear_q), and with
+    the oracle. `pad` widens the row stride so float4 loads are ruled out."""
+    x, w, b = _case(m, k, n, seed=1000 + m)
+    if m > 2:
+        x[2] = 0.0
+    xbuf = np.zeros((m, k + pad), np.float32)
+    xbuf[:, :k] = x
+    xd = dev(xbuf)[:, :k]
+    wp, sw = oracle.w4_quantize_pack(w)
+    wpd, swd, bd = dev(wp), dev(sw), dev(b)
+    y1 = nat.w4a8_linear(xd, wpd, swd, bias=bd, path="decode")
+    xq, sx = nat.a8_quantize_rows(xd)
+    y2 = nat.w4a8_linear_q(xq, sx, k, wpd, swd, bias=bd, path="decode")
+    a, c = host(y1), host(y2)
+    assert np.array_equal(a.view(np.uint32), c.view(np.uint32))
+    assert_f32_close(a, oracle.linear(x, wp, sw, k, bias=b), b)

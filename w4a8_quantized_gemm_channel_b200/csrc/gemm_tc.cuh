@@ -36,13 +36,18 @@ namespace tc {
 constexpr int BM = 128;            // output channels per tile (MMA M)
 constexpr int BK = 128;            // k per stage
 constexpr int MMA_K = 32;          // k per kind::i8 instruction
-// 6 stages: 144 KB of shared memory, which also keeps a second CTA (that
-// would block in tcgen05.alloc of the whole TMEM) off the SM.
-constexpr int STAGES = 6;
-// Unpack warpgroups: stage s is unpacked by warpgroup s % UNPACK_WG, so the
-// groups overlap their shared-memory reads, integer work and TMEM stores.
+// Two rings. Shared-memory stages (TMA -> unpack/MMA) are deep, so loads run
+// far ahead of the tensor pipe: 8 x 24 KB = 192 KB, which also keeps a second
+// CTA (that would block in tcgen05.alloc of the whole TMEM) off the SM. TMEM A
+// slots (unpack -> MMA) only cover the short unpack hop: 6 x 32 columns next
+// to the two 128-column accumulators.
+constexpr int STAGES = 8;
+constexpr int A_SLOTS = 6;
+// Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
+// it % UNPACK_WG, so the groups overlap their shared-memory reads, integer
+// work and TMEM stores.
 constexpr int UNPACK_WG = 3;
-static_assert(STAGES % UNPACK_WG == 0, "each warpgroup owns fixed ring slots");
+static_assert(A_SLOTS % UNPACK_WG == 0, "each warpgroup owns fixed TMEM slots");
 constexpr int FIRST_UNPACK_WARP = 4;
 constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + 4 * UNPACK_WG;
 constexpr int NUM_THREADS = 32 * (FIRST_EPI_WARP + 4);
@@ -55,27 +60,43 @@ struct alignas(1024) Smem {
     uint8_t act[STAGES][BT * BK];        // activation tiles, 128B-swizzled rows
     uint8_t wpk[STAGES][W_TILE_BYTES];   // packed weight tiles, 64B-swizzled rows
     uint64_t full[STAGES];               // TMA landed (tx-count barrier)
-    uint64_t aready[STAGES];             // A slot written to TMEM (4 unpack warps)
     uint64_t empty[STAGES];              // MMAs reading the stage finished
+    uint64_t aready[A_SLOTS];            // A slot written to TMEM (4 unpack warps)
+    uint64_t afree[A_SLOTS];             // MMAs reading the A slot finished
     uint64_t acc_full[2];                // accumulator ready for the epilogue
     uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
     uint64_t mma_done;                   // final drain of the MMA pipe
     float rsx[BT];                       // 1/sx of the epilogue's current token tile
+    float tsx[BT];                       // sx of the same tokens
     uint32_t tmem_base;
     int abort;
 };
 
+// How the weight warpgroups widen nibbles to the INT8 A operand.
+//  UNPACK_SEXT: sign-extend each nibble (byte = q), then restore k order with
+//      two byte permutes. Any K.
+//  UNPACK_X16:  keep each nibble in the high half of its byte, so the byte is
+//      exactly 16*q as INT8 (q in [-8, 7] gives 16q in [-128, 112]); the
+//      accumulator is then exactly 16*acc and the epilogue shifts it back.
+//      Two masks and one shift per 8 codes, plus the two byte permutes.
+//      Needs 16 * 128 * 127 * K < 2^31, i.e. K <= TC_X16_MAX_K.
+//  UNPACK_X16_PERM: as UNPACK_X16 without the byte permutes: the activations
+//      were stored with each group of 8 k reordered to k0 k2 k4 k6 k1 k3 k5 k7
+//      (see k_act_quant), which is the order the masks produce.
+enum { UNPACK_SEXT = 0, UNPACK_X16 = 1, UNPACK_X16_PERM = 2 };
+constexpr int TC_X16_MAX_K = 131072;
+
 template <int BT>
 constexpr int d_col(int buf) { return buf * BT; }
 template <int BT>
-constexpr int a_col(int stage) { return 2 * BT + stage * A_COLS; }
+constexpr int a_col(int slot) { return 2 * BT + slot * A_COLS; }
 
-template <int BT>
+template <int BT, int UNPACK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
           int M, int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
           const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
-    static_assert(2 * BT + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+    static_assert(2 * BT + A_SLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
     extern __shared__ uint8_t smem_raw[];
     Smem<BT> &sm = *reinterpret_cast<Smem<BT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,8 +110,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             ptx::mbar_init(&sm.full[s], 1);
-            ptx::mbar_init(&sm.aready[s], 4);
             ptx::mbar_init(&sm.empty[s], 1);
+        }
+        for (int a = 0; a < A_SLOTS; ++a) {
+            ptx::mbar_init(&sm.aready[a], 4);
+            ptx::mbar_init(&sm.afree[a], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&sm.acc_full[b], 1);
@@ -148,6 +172,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             constexpr uint32_t idesc = ptx::idesc_i8(BM, BT);
             int stage = 0;
             uint32_t phase = 0;
+            int slot = 0;
+            uint32_t aphase = 0;
             int buf = 0;
             uint32_t acc_phase = 0;
             bool ok = true, any = false;
@@ -157,9 +183,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 const uint32_t d = tmem + (uint32_t)d_col<BT>(buf);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!ptx::mbar_wait(&sm.full[stage], phase, abort) ||
-                        !ptx::mbar_wait(&sm.aready[stage], phase, abort)) { ok = false; break; }
+                        !ptx::mbar_wait(&sm.aready[slot], aphase, abort)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    const uint32_t a = tmem + (uint32_t)a_col<BT>(stage);
+                    const uint32_t a = tmem + (uint32_t)a_col<BT>(slot);
                     const uint32_t b = ptx::smem_addr(sm.act[stage]);
 #pragma unroll
                     for (int kk = 0; kk < BK / MMA_K; ++kk) {
@@ -168,7 +194,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                     }
                     any = true;
                     ptx::mma_commit(&sm.empty[stage]);
+                    ptx::mma_commit(&sm.afree[slot]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (++slot == A_SLOTS) { slot = 0; aphase ^= 1; }
                 }
                 if (!ok) break;
                 ptx::mma_commit(&sm.acc_full[buf]);
@@ -191,20 +219,21 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
         const int wg = (warp - FIRST_UNPACK_WARP) >> 2;
         const int r = q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        int stage = 0;
-        uint32_t phase = 0;
         bool ok = true;
-        int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                if (it % UNPACK_WG != wg) {
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    continue;
-                }
+        int it = wg;  // this warpgroup's iterations: wg, wg + UNPACK_WG, ...
+        const int total = ((num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * num_kb;
+        for (; it < total && ok; it += UNPACK_WG) {
+            {
+                const int stage = it % STAGES;
+                const uint32_t phase = (uint32_t)(it / STAGES) & 1u;
+                const int slot = it % A_SLOTS;
+                const uint32_t aphase = (uint32_t)(it / A_SLOTS) & 1u;
                 // every lane waits (each then sees the TMA data); the outcome is
                 // made warp-uniform before the warp-collective tcgen05.st
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sm.full[stage], phase, abort));
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sm.full[stage], phase, abort) &&
+                                                 ptx::mbar_wait(&sm.afree[slot], aphase ^ 1, abort));
                 if (!ok) break;
+                ptx::tc_fence_after();
                 const uint8_t *row = sm.wpk[stage] + r * (BK / 2);
                 const int sx_ = (r >> 1) & 3;
                 uint32_t out[32];
@@ -214,18 +243,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                     const uint32_t p[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        uint32_t lo, hi;
-                        unpack_s4x8(p[j], lo, hi);  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
-                        out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
-                        out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                        uint32_t lo, hi;  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
+                        if constexpr (UNPACK == UNPACK_SEXT) {
+                            unpack_s4x8(p[j], lo, hi);
+                        } else {
+                            lo = (p[j] << 4) & 0xF0F0F0F0u;
+                            hi = p[j] & 0xF0F0F0F0u;
+                        }
+                        if constexpr (UNPACK == UNPACK_X16_PERM) {
+                            out[8 * c + 2 * j] = lo;
+                            out[8 * c + 2 * j + 1] = hi;
+                        } else {
+                            out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
+                            out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                        }
                     }
                 }
-                ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)a_col<BT>(stage), out);
+                ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)a_col<BT>(slot), out);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sm.aready[stage]);
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                if (lane == 0) ptx::mbar_arrive(&sm.aready[slot]);
             }
         }
     } else if (warp >= FIRST_EPI_WARP) {
@@ -254,7 +292,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             // readers are past the named barrier at its end)
             for (int c = et; c < BT; c += 128) {
                 const int m = m_base + c;
-                sm.rsx[c] = m < M ? __frcp_rn(__ldg(sx + m)) : 0.0f;
+                const float v = m < M ? __ldg(sx + m) : 1.0f;
+                sm.tsx[c] = v;
+                sm.rsx[c] = __frcp_rn(v);
             }
             // One decision for all four epilogue warps (this barrier also
             // publishes rsx): a warp that gave up must not leave the others
@@ -278,12 +318,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                     if (j < mrem && n_ok) {
                         const int m = m_base + c0 + j;
                         const size_t off = (size_t)m * (size_t)ldy + (size_t)n;
-                        const int32_t acc = (int32_t)v[j];
+                        const int32_t acc = UNPACK == UNPACK_SEXT ? (int32_t)v[j] : ((int32_t)v[j] >> 4);
                         if (fmt == W4A8_OUT_S32) {
                             static_cast<int32_t *>(Y)[off] = acc;
                         } else {
                             const float f = __int2float_rn(acc);
-                            const float d = __fmul_rn(__ldg(sx + m), swn);
+                            const float d = __fmul_rn(sm.tsx[c0 + j], swn);
                             const float r = __fmul_rn(sm.rsx[c0 + j], rswn);
                             const float q0 = __fmul_rn(f, r);
                             const float e = __fmaf_rn(-q0, d, f);
@@ -349,14 +389,14 @@ inline bool make_map_u8(CUtensorMap *map, const void *base, uint64_t inner, uint
 template <int BT>
 inline size_t smem_bytes() { return sizeof(Smem<BT>) + 1024; }
 
-template <int BT>
+template <int BT, int UNPACK>
 inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
                           const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy, int sm_count,
                           cudaStream_t stream) {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(k_gemm_tc<BT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(k_gemm_tc<BT, UNPACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)smem_bytes<BT>());
     });
     if (attr_err != cudaSuccess) return W4A8_ERR_CUDA;
@@ -377,7 +417,7 @@ inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_tc<BT>, tm_w, tm_x, M, N, K, sx, sw, bias, flags, Y, ldy);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_tc<BT, UNPACK>, tm_w, tm_x, M, N, K, sx, sw, bias, flags, Y, ldy);
     return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
@@ -387,10 +427,21 @@ inline bool tc_supported(int M, int K, int N) {
     return M >= 1 && K >= 1 && N >= 1 && tc::encode_fn() != nullptr;
 }
 
+// act_perm: the INT8 activations use the k-permuted layout k_act_quant
+// writes for this kernel (only inside w4a8_linear's workspace).
 inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp,
                                   int ldp, const float *sw, int N, const float *bias, unsigned flags, void *Y,
-                                  int ldy, int sm_count, cudaStream_t stream) {
-    return tc::launch<128>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+                                  int ldy, int sm_count, cudaStream_t stream, bool act_perm = false) {
+    if (K > tc::TC_X16_MAX_K) {
+        if (act_perm) return W4A8_ERR_UNSUPPORTED;
+        return tc::launch<128, tc::UNPACK_SEXT>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
+                                                stream);
+    }
+    if (act_perm)
+        return tc::launch<128, tc::UNPACK_X16_PERM>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+                                                    sm_count, stream);
+    return tc::launch<128, tc::UNPACK_X16>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
+                                           stream);
 }
 
 }  // namespace w4a8

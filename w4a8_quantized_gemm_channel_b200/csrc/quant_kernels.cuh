@@ -101,26 +101,28 @@ k_quant_pack(const float *__restrict__ W, int K, int N, int ldw,
     float s[VEC];
 #pragma unroll
     for (int c = 0; c < VEC; ++c) s[c] = (n + c < N) ? weight_scale_from_amax(__ldg(amax_bits + n + c)) : 1.0f;
+    // all eight rows of this thread in flight before any of them is used
+    float v[8][VEC];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int kk = warp + 8 * i;
-        const int k = k0 + kk;
-        float v[VEC];
+        const int k = k0 + warp + 8 * i;
         if (k < K && n < N) {
             if constexpr (VEC == 4) {
                 const float4 f = __ldg(reinterpret_cast<const float4 *>(W + (size_t)k * ldw + n));
-                v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+                v[i][0] = f.x; v[i][1] = f.y; v[i][2] = f.z; v[i][3] = f.w;
             } else {
-                v[0] = __ldg(W + (size_t)k * ldw + n);
+                v[i][0] = __ldg(W + (size_t)k * ldw + n);
             }
         } else {
 #pragma unroll
-            for (int c = 0; c < VEC; ++c) v[c] = 0.0f;
+            for (int c = 0; c < VEC; ++c) v[i][c] = 0.0f;
         }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int c = 0; c < VEC; ++c)
-            qs[lane * VEC + c][kk] = (int8_t)clampi(__float2int_rn(__fmul_rn(v[c], s[c])), -8, 7);
-    }
+            qs[lane * VEC + c][warp + 8 * i] = (int8_t)clampi(__float2int_rn(__fmul_rn(v[i][c], s[c])), -8, 7);
     __syncthreads();
     // 2 threads per output channel row, 16 packed bytes (32 codes) each.
     for (int tt = threadIdx.x; tt < 2 * COLS; tt += 256) {
@@ -153,14 +155,65 @@ __global__ void k_weight_scale_finalize(float *__restrict__ sw, int N) {
 // Activation quantization: one block per row (grid-stride over rows).
 // The row is read once into registers (VPT floats per thread; longer rows
 // are re-read for the quantization pass), its abs-max reduced with warp
-// shuffles and then across warps, and the codes leave 4 per 32-bit store.
+// shuffles and then across warps, and the codes are stored 4 (or 8) at a time.
 // Bytes K..ldq-1 of each row are written 0.
+//
+// PERM = false: natural k order (the public layout of a8_quantize_rows).
+// PERM = true: inside every group of 8 consecutive k the bytes are stored as
+// k0 k2 k4 k6 k1 k3 k5 k7 - the order in which the tensor-core kernel's
+// weight unpack produces codes - so that kernel needs no byte permutes. Only
+// used for the INT8 activations w4a8_linear keeps in its workspace.
 // ---------------------------------------------------------------------------
-template <int THREADS, int VPT>
+__device__ __forceinline__ float row_load(const float *__restrict__ x, int k, int K) {
+    return k < K ? __ldg(x + k) : 0.0f;
+}
+
+template <int U>
+__device__ __forceinline__ void load_unit(const float *__restrict__ x, int k, int K, bool vec4, float (&v)[U]) {
+#pragma unroll
+    for (int h = 0; h < U / 4; ++h) {
+        const int kk = k + 4 * h;
+        if (vec4 && kk + 3 < K) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(x + kk));
+            v[4 * h] = f.x; v[4 * h + 1] = f.y; v[4 * h + 2] = f.z; v[4 * h + 3] = f.w;
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) v[4 * h + b] = row_load(x, kk + b, K);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t code8(float v, float s, bool in) {
+    const int q = in ? clampi(__float2int_rn(__fmul_rn(v, s)), -127, 127) : 0;
+    return (uint32_t)(q & 0xFF);
+}
+
+// Quantize one unit of U consecutive k (k0 = first k) and store it.
+template <int U, bool PERM>
+__device__ __forceinline__ void store_unit(int8_t *__restrict__ row, int k0, int K, float s, const float (&v)[U]) {
+    if constexpr (!PERM) {
+        uint32_t w = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) w |= code8(v[b], s, k0 + b < K) << (8 * b);
+        *reinterpret_cast<uint32_t *>(row + k0) = w;
+    } else {
+        uint32_t even = 0, odd = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            even |= code8(v[2 * b], s, k0 + 2 * b < K) << (8 * b);
+            odd |= code8(v[2 * b + 1], s, k0 + 2 * b + 1 < K) << (8 * b);
+        }
+        *reinterpret_cast<uint2 *>(row + k0) = make_uint2(even, odd);
+    }
+}
+
+template <int THREADS, int VPT, bool PERM>
 __global__ void __launch_bounds__(THREADS)
 k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
             int8_t *__restrict__ Xq, int ldq, float *__restrict__ sx, int vec4) {
-    static_assert(THREADS % 32 == 0 && THREADS <= 1024 && VPT % 4 == 0, "block shape");
+    constexpr int U = PERM ? 8 : 4;  // consecutive k per unit of work
+    constexpr int G = VPT / U;       // units a thread keeps in registers
+    static_assert(THREADS % 32 == 0 && THREADS <= 1024 && VPT % U == 0, "block shape");
     __shared__ float red[THREADS / 32];
     // Let the next kernel launch now: it only prefetches weights before its
     // own griddepcontrol.wait, which returns after this grid has finished.
@@ -169,26 +222,19 @@ k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
     griddep_launch_dependents();
     griddep_wait();  // X may be written by the previous kernel
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // Thread j of the block owns the 4-element groups j, j + THREADS, ...
-    constexpr int G = VPT / 4;
     const bool in_regs = K <= THREADS * VPT;
+    const int units = ldq / U;  // ldq is a multiple of 16
     for (int m = blockIdx.x; m < M; m += gridDim.x) {
         const float *x = X + (size_t)m * ldx;
-        float v[G][4];
+        // unit u covers k = U*u .. U*u + U-1; thread t holds units t + i*THREADS
+        float v[G][U];
         float amax = 0.0f;
         if (in_regs) {
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-                const int k = 4 * (threadIdx.x + gi * THREADS);
-                if (vec4 && k + 3 < K) {
-                    const float4 f = __ldg(reinterpret_cast<const float4 *>(x + k));
-                    v[gi][0] = f.x; v[gi][1] = f.y; v[gi][2] = f.z; v[gi][3] = f.w;
-                } else {
+            for (int i = 0; i < G; ++i) {
+                load_unit<U>(x, U * (threadIdx.x + i * THREADS), K, vec4 != 0, v[i]);
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) v[gi][b] = (k + b < K) ? __ldg(x + k + b) : 0.0f;
-                }
-#pragma unroll
-                for (int b = 0; b < 4; ++b) amax = fmaxf(amax, fabsf(v[gi][b]));
+                for (int b = 0; b < U; ++b) amax = fmaxf(amax, fabsf(v[i][b]));
             }
         } else {
             for (int k = threadIdx.x; k < K; k += THREADS) amax = fmaxf(amax, fabsf(__ldg(x + k)));
@@ -202,32 +248,24 @@ k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
         for (int i = 1; i < THREADS / 32; ++i) a = fmaxf(a, red[i]);
         const float s = a == 0.0f ? 1.0f : __fdiv_rn(127.0f, a);
         if (threadIdx.x == 0) sx[m] = s;
-        uint32_t *q4 = reinterpret_cast<uint32_t *>(Xq + (size_t)m * ldq);
+        int8_t *row = Xq + (size_t)m * ldq;
         if (in_regs) {
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-                const int j = threadIdx.x + gi * THREADS;
-                if (4 * j < ldq) {
-                    uint32_t packed = 0;
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const int q = (4 * j + b < K) ? clampi(__float2int_rn(__fmul_rn(v[gi][b], s)), -127, 127) : 0;
-                        packed |= (uint32_t)(q & 0xFF) << (8 * b);
-                    }
-                    q4[j] = packed;
-                }
+            for (int i = 0; i < G; ++i) {
+                const int u = threadIdx.x + i * THREADS;
+                if (u < units) store_unit<U, PERM>(row, U * u, K, s, v[i]);
             }
-            for (int j = threadIdx.x + G * THREADS; j < ldq / 4; j += THREADS) q4[j] = 0;
-        } else {
-            for (int j = threadIdx.x; j < ldq / 4; j += THREADS) {
-                uint32_t packed = 0;
+            for (int u = threadIdx.x + G * THREADS; u < units; u += THREADS) {
+                float z[U];
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int k = 4 * j + b;
-                    const int q = (k < K) ? clampi(__float2int_rn(__fmul_rn(__ldg(x + k), s)), -127, 127) : 0;
-                    packed |= (uint32_t)(q & 0xFF) << (8 * b);
-                }
-                q4[j] = packed;
+                for (int b = 0; b < U; ++b) z[b] = 0.0f;
+                store_unit<U, PERM>(row, U * u, K, s, z);
+            }
+        } else {
+            for (int u = threadIdx.x; u < units; u += THREADS) {
+                float w[U];
+                load_unit<U>(x, U * u, K, vec4 != 0, w);
+                store_unit<U, PERM>(row, U * u, K, s, w);
             }
         }
         __syncthreads();  // red is reused by the next row

@@ -118,13 +118,15 @@ unsigned choose_path(int M, int K, int N, unsigned flags) {
     return W4A8_PATH_DECODE;
 }
 
+// act_perm: Xq uses the k-permuted layout (only the tensor-core path reads it).
 w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx,
                         const uint8_t *Wp, int ldp, const float *sw, int N,
                         const float *bias, unsigned flags, void *Y, int ldy,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, bool act_perm = false) {
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
     const unsigned path = choose_path(M, K, N, flags);
+    if (act_perm && path != W4A8_PATH_TC) return W4A8_ERR_INVALID_ARG;
     cudaError_t e = cudaSuccess;
     if (path == W4A8_PATH_GENERIC) {
         dim3 grid((N + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
@@ -144,7 +146,7 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     } else if (path == W4A8_PATH_TC) {
         if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
         w4a8_status st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
-                                        dev.sm_count, stream);
+                                        dev.sm_count, stream, act_perm);
         if (st != W4A8_OK) return st;
     } else {
         return W4A8_ERR_INVALID_ARG;
@@ -230,15 +232,34 @@ w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp,
 }
 
 static w4a8_status launch_act_quant(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
-                                    float *sx, cudaStream_t s) {
+                                    float *sx, cudaStream_t s, bool perm = false) {
     const int vec4 = aligned16(X) && (ldx % 4 == 0);
     const int grid = M < 65535 ? M : 65535;
     cudaError_t e;
-    if (K <= 1024)
-        e = launch_pdl(k_act_quant<128, 8>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
-    else
-        e = launch_pdl(k_act_quant<256, 16>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+    if (perm) {
+        if (K <= 1024)
+            e = launch_pdl(k_act_quant<128, 8, true>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+        else
+            e = launch_pdl(k_act_quant<256, 16, true>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+    } else {
+        if (K <= 1024)
+            e = launch_pdl(k_act_quant<128, 8, false>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+        else
+            e = launch_pdl(k_act_quant<256, 16, false>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+    }
     return from_cuda(e);
+}
+
+// Steps 3-6 on float32 activations with the INT8 copy in `ws`: the path is
+// chosen first, so the tensor-core GEMM gets its k-permuted activation layout.
+static w4a8_status linear_from_f32(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp,
+                                   const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                                   const Workspace &ws, cudaStream_t s) {
+    const unsigned path = choose_path(M, K, N, flags);
+    const bool perm = path == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
+    w4a8_status st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s, perm);
+    if (st != W4A8_OK) return st;
+    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s, perm);
 }
 
 w4a8_status a8_quantize_rows(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
@@ -263,10 +284,8 @@ w4a8_status w4a8_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp
     if (workspace_bytes < w4a8_workspace_size(M, K)) return W4A8_ERR_WORKSPACE;
     if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
     const Workspace ws = carve_workspace(workspace, M, K);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
-    if (st != W4A8_OK) return st;
-    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
+    return linear_from_f32(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, ws,
+                           static_cast<cudaStream_t>(stream));
 }
 
 w4a8_status w4a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
@@ -294,10 +313,8 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
     void *scratch = noalloc_scratch_ptr();
     if (!scratch) return W4A8_ERR_CUDA;
     const Workspace ws = carve_workspace(scratch, M, K);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
-    if (st != W4A8_OK) return st;
-    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
+    return linear_from_f32(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, ws,
+                           static_cast<cudaStream_t>(stream));
 }
 
 unsigned w4a8_last_path(void) { return t_last_path; }
