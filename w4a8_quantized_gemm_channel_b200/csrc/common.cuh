@@ -30,6 +30,53 @@ __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Loads of values that a grid this launch depends on may write (activations,
+// scales, bias; the weights too, as far as the kernel can tell). The kernels
+// here are launched with a programmatic dependency, so they can be running
+// while their predecessor still writes: such values are not constant for the
+// kernel's lifetime, which the read-only (.nc, __ldg) path requires, and a
+// load the compiler treats as invariant may be scheduled above
+// griddepcontrol.wait. These are plain coherent loads in volatile asm, which
+// stays in program order with the (volatile) wait.
+//   ld_dep*   : cached at all levels (reused operands);
+//   ld_dep_cg*: cached in L2 only, for bytes that are used once.
+__device__ __forceinline__ float ld_dep(const float *p) {
+    float v;
+    asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_dep_u8(const uint8_t *p) {
+    uint32_t v;
+    asm volatile("ld.global.u8 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ int32_t ld_dep_s8(const int8_t *p) {
+    int32_t v;
+    asm volatile("ld.global.s8 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float4 ld_dep_f4(const float *p) {
+    float4 v;
+    asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_dep_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_dep_cg_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 // Warm L2 with [p, p + bytes) (bytes a multiple of 16, p 16-byte aligned)
 // without returning data: safe to issue before griddepcontrol.wait, because
 // L2 is the point of coherence and no stale value reaches a register.
@@ -58,7 +105,7 @@ __device__ __forceinline__ float dequant_one(int32_t acc, float sxm, float swn,
                                              bool relu) {
     float d = __fmul_rn(sxm, swn);
     float y = __fdiv_rn(__int2float_rn(acc), d);
-    if (bias) y = __fadd_rn(y, bias[n]);
+    if (bias) y = __fadd_rn(y, ld_dep(bias + n));
     if (relu) y = y > 0.0f ? y : 0.0f;
     return y;
 }

@@ -48,6 +48,10 @@ constexpr int A_SLOTS = 6;
 // work and TMEM stores.
 constexpr int UNPACK_WG = 3;
 static_assert(A_SLOTS % UNPACK_WG == 0, "each warpgroup owns fixed TMEM slots");
+// The unpack warps reuse A slot it % A_SLOTS once the stage barrier of
+// iteration it - A_SLOTS has flipped; that barrier is not reused before
+// iteration it - A_SLOTS + STAGES >= it, which cannot have run yet.
+static_assert(STAGES >= A_SLOTS, "A-slot reuse waits on a stage barrier");
 constexpr int FIRST_UNPACK_WARP = 4;
 constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + 4 * UNPACK_WG;
 constexpr int NUM_THREADS = 32 * (FIRST_EPI_WARP + 4);
@@ -62,7 +66,6 @@ struct alignas(1024) Smem {
     uint64_t full[STAGES];               // TMA landed (tx-count barrier)
     uint64_t empty[STAGES];              // MMAs reading the stage finished
     uint64_t aready[A_SLOTS];            // A slot written to TMEM (4 unpack warps)
-    uint64_t afree[A_SLOTS];             // MMAs reading the A slot finished
     uint64_t acc_full[2];                // accumulator ready for the epilogue
     uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
     uint64_t mma_done;                   // final drain of the MMA pipe
@@ -91,6 +94,52 @@ constexpr int d_col(int buf) { return buf * BT; }
 template <int BT>
 constexpr int a_col(int slot) { return 2 * BT + slot * A_COLS; }
 
+// Epilogue of one 32-token chunk for one output channel (this thread's TMEM
+// lane): dequantize, bias, ReLU, store. Every choice is a template argument so
+// the unrolled loop holds no branches (runtime branches per element made this
+// loop several times slower); a chunk cut by the end of M takes the predicated
+// form. v = raw TMEM words, SHIFT = 4 when they hold 16*acc.
+enum { EPI_F32 = 0, EPI_BF16 = 1, EPI_S32 = 2 };
+
+template <int FMT, bool BIAS, bool RELU, int SHIFT, bool FULL>
+__device__ __forceinline__ void epi_chunk(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0, int mrem,
+                                          int n, bool n_ok, float swn, float rswn, float bn,
+                                          const float *__restrict__ tsx, const float *__restrict__ rsx) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (!FULL && j >= mrem) break;
+        const int32_t acc = (int32_t)v[j] >> SHIFT;
+        const size_t off = (size_t)(m0 + j) * (size_t)ldy + (size_t)n;
+        if constexpr (FMT == EPI_S32) {
+            if (n_ok) static_cast<int32_t *>(Y)[off] = acc;
+        } else {
+            const float f = __int2float_rn(acc);
+            const float d = __fmul_rn(tsx[j], swn);
+            const float r = __fmul_rn(rsx[j], rswn);
+            const float q0 = __fmul_rn(f, r);
+            const float e = __fmaf_rn(-q0, d, f);
+            float y = __fmaf_rn(e, r, q0);
+            if constexpr (BIAS) y = __fadd_rn(y, bn);
+            if constexpr (RELU) y = y > 0.0f ? y : 0.0f;
+            if constexpr (FMT == EPI_BF16) {
+                if (n_ok) static_cast<__nv_bfloat16 *>(Y)[off] = __float2bfloat16_rn(y);
+            } else {
+                if (n_ok) static_cast<float *>(Y)[off] = y;
+            }
+        }
+    }
+}
+
+template <int FMT, bool BIAS, bool RELU, int SHIFT>
+__device__ __forceinline__ void epi_chunk_any(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0,
+                                              int mrem, int n, bool n_ok, float swn, float rswn, float bn,
+                                              const float *__restrict__ tsx, const float *__restrict__ rsx) {
+    if (mrem >= 32)
+        epi_chunk<FMT, BIAS, RELU, SHIFT, true>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx);
+    else
+        epi_chunk<FMT, BIAS, RELU, SHIFT, false>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx);
+}
+
 template <int BT, int UNPACK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
@@ -112,10 +161,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             ptx::mbar_init(&sm.full[s], 1);
             ptx::mbar_init(&sm.empty[s], 1);
         }
-        for (int a = 0; a < A_SLOTS; ++a) {
-            ptx::mbar_init(&sm.aready[a], 4);
-            ptx::mbar_init(&sm.afree[a], 1);
-        }
+        for (int a = 0; a < A_SLOTS; ++a) ptx::mbar_init(&sm.aready[a], 4);
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&sm.acc_full[b], 1);
             ptx::mbar_init(&sm.acc_empty[b], 4);
@@ -168,39 +214,58 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
         }
     } else if (warp == 1) {
         // ---------------------------------------------------- MMA issuer
+        // One iteration = one stage (BK k) of one tile: 4 MMAs into the tile's
+        // accumulator, then one commit that frees the shared-memory stage (and,
+        // A_SLOTS iterations later, the TMEM A slot: the unpack warps wait on the
+        // same barrier). The tensor core queues only about one MMA ahead, so the
+        // waits for the next iteration's operands are done before the last MMA
+        // of this one is issued, while the queued MMAs still run.
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_i8(BM, BT);
-            int stage = 0;
-            uint32_t phase = 0;
-            int slot = 0;
-            uint32_t aphase = 0;
-            int buf = 0;
-            uint32_t acc_phase = 0;
-            bool ok = true, any = false;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                if (!ptx::mbar_wait(&sm.acc_empty[buf], acc_phase ^ 1, abort)) { ok = false; break; }
+            constexpr int KSTEPS = BK / MMA_K;
+            const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+            const int total = my_tiles * num_kb;
+            // ring positions of the current iteration (incremental: no divisions
+            // on this thread, which paces the tensor core)
+            int stage = 0, slot = 0, kb = 0, buf = 0;
+            uint32_t sphase = 0, aphase = 0, bphase = 0;
+            // the unpack warps signal aready only after their own wait on
+            // full[], so the TMA data of that iteration has landed as well
+            bool ok = total > 0 ? (ptx::mbar_wait(&sm.full[0], 0, abort) && ptx::mbar_wait(&sm.aready[0], 0, abort))
+                                : true;
+            bool any = false;
+            for (int it = 0; it < total && ok; ++it) {
+                if (kb == 0) {
+                    if (!ptx::mbar_wait(&sm.acc_empty[buf], bphase ^ 1u, abort)) break;
+                }
                 ptx::tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)d_col<BT>(buf);
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!ptx::mbar_wait(&sm.full[stage], phase, abort) ||
-                        !ptx::mbar_wait(&sm.aready[slot], aphase, abort)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t a = tmem + (uint32_t)a_col<BT>(slot);
-                    const uint32_t b = ptx::smem_addr(sm.act[stage]);
+                const uint32_t a = tmem + (uint32_t)a_col<BT>(slot);
+                const uint32_t b = ptx::smem_addr(sm.act[stage]);
 #pragma unroll
-                    for (int kk = 0; kk < BK / MMA_K; ++kk) {
-                        ptx::mma_i8_ts(d, a + kk * (MMA_K / 4), ptx::sdesc_k_sw128(b + kk * MMA_K), idesc,
-                                       (kb | kk) != 0);
-                    }
-                    any = true;
-                    ptx::mma_commit(&sm.empty[stage]);
-                    ptx::mma_commit(&sm.afree[slot]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    if (++slot == A_SLOTS) { slot = 0; aphase ^= 1; }
+                for (int kk = 0; kk < KSTEPS - 1; ++kk)
+                    ptx::mma_i8_ts(d, a + kk * (MMA_K / 4), ptx::sdesc_k_sw128(b + kk * MMA_K), idesc,
+                                   (kb | kk) != 0);
+                // next ring positions; wait for their operands while the MMAs
+                // already queued keep the tensor core busy
+                int nstage = stage + 1, nslot = slot + 1;
+                uint32_t nsphase = sphase, naphase = aphase;
+                if (nstage == STAGES) { nstage = 0; nsphase ^= 1u; }
+                if (nslot == A_SLOTS) { nslot = 0; naphase ^= 1u; }
+                const bool next_ok = it + 1 < total ? (ptx::mbar_wait(&sm.full[nstage], nsphase, abort) &&
+                                                       ptx::mbar_wait(&sm.aready[nslot], naphase, abort))
+                                                    : true;
+                ptx::mma_i8_ts(d, a + (KSTEPS - 1) * (MMA_K / 4), ptx::sdesc_k_sw128(b + (KSTEPS - 1) * MMA_K),
+                               idesc, 1u);
+                any = true;
+                ptx::mma_commit(&sm.empty[stage]);
+                if (++kb == num_kb) {
+                    ptx::mma_commit(&sm.acc_full[buf]);
+                    kb = 0;
+                    if (++buf == 2) { buf = 0; bphase ^= 1u; }
                 }
-                if (!ok) break;
-                ptx::mma_commit(&sm.acc_full[buf]);
-                if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+                stage = nstage; sphase = nsphase; slot = nslot; aphase = naphase;
+                ok = next_ok;
             }
             if (any) {
                 // All MMAs done before TMEM is released.
@@ -230,8 +295,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 const uint32_t aphase = (uint32_t)(it / A_SLOTS) & 1u;
                 // every lane waits (each then sees the TMA data); the outcome is
                 // made warp-uniform before the warp-collective tcgen05.st
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait(&sm.full[stage], phase, abort) &&
-                                                 ptx::mbar_wait(&sm.afree[slot], aphase ^ 1, abort));
+                // the slot was last read by iteration it - A_SLOTS, whose MMAs
+                // completed when that iteration's stage barrier flipped
+                bool got = ptx::mbar_wait(&sm.full[stage], phase, abort);
+                if (got && it >= A_SLOTS) {
+                    const int j = it - A_SLOTS;
+                    got = ptx::mbar_wait(&sm.empty[j % STAGES], (uint32_t)(j / STAGES) & 1u, abort);
+                }
+                (void)aphase;
+                ok = __all_sync(0xffffffffu, got);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint8_t *row = sm.wpk[stage] + r * (BK / 2);
@@ -284,7 +356,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
         int buf = 0;
         uint32_t acc_phase = 0;
         const unsigned fmt = flags & W4A8_OUT_MASK;
-        const bool relu = (flags & W4A8_RELU) != 0;
+        const int epi_mode = fmt == W4A8_OUT_S32 ? 8
+                             : (fmt == W4A8_OUT_BF16 ? 4 : 0) + (bias ? 2 : 0) + ((flags & W4A8_RELU) ? 1 : 0);
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int n_tile = tile / tiles_m, m_tile = tile % tiles_m;
             const int m_base = m_tile * BT;
@@ -292,7 +365,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             // readers are past the named barrier at its end)
             for (int c = et; c < BT; c += 128) {
                 const int m = m_base + c;
-                const float v = m < M ? __ldg(sx + m) : 1.0f;
+                const float v = m < M ? ld_dep(sx + m) : 1.0f;
                 sm.tsx[c] = v;
                 sm.rsx[c] = __frcp_rn(v);
             }
@@ -303,9 +376,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             ptx::tc_fence_after();
             const int n = n_tile * BM + q * 32 + lane;
             const bool n_ok = n < N;
-            const float swn = n_ok ? __ldg(sw + n) : 1.0f;
+            const float swn = n_ok ? ld_dep(sw + n) : 1.0f;
             const float rswn = __frcp_rn(swn);
-            const float bn = (bias && n_ok) ? __ldg(bias + n) : 0.0f;
+            const float bn = (bias && n_ok) ? ld_dep(bias + n) : 0.0f;
 #pragma unroll 1
             for (int c0 = 0; c0 < BT; c0 += 32) {
                 uint32_t v[32];
@@ -313,30 +386,22 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 ptx::tmem_wait_ld();
                 const int mrem = M - (m_base + c0);
                 if (mrem <= 0) break;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    if (j < mrem && n_ok) {
-                        const int m = m_base + c0 + j;
-                        const size_t off = (size_t)m * (size_t)ldy + (size_t)n;
-                        const int32_t acc = UNPACK == UNPACK_SEXT ? (int32_t)v[j] : ((int32_t)v[j] >> 4);
-                        if (fmt == W4A8_OUT_S32) {
-                            static_cast<int32_t *>(Y)[off] = acc;
-                        } else {
-                            const float f = __int2float_rn(acc);
-                            const float d = __fmul_rn(sm.tsx[c0 + j], swn);
-                            const float r = __fmul_rn(sm.rsx[c0 + j], rswn);
-                            const float q0 = __fmul_rn(f, r);
-                            const float e = __fmaf_rn(-q0, d, f);
-                            float y = __fmaf_rn(e, r, q0);
-                            if (bias) y = __fadd_rn(y, bn);
-                            if (relu) y = y > 0.0f ? y : 0.0f;
-                            if (fmt == W4A8_OUT_BF16)
-                                static_cast<__nv_bfloat16 *>(Y)[off] = __float2bfloat16_rn(y);
-                            else
-                                static_cast<float *>(Y)[off] = y;
-                        }
-                    }
+                constexpr int SH = UNPACK == UNPACK_SEXT ? 0 : 4;
+                const int m0 = m_base + c0;
+                const float *tsx = sm.tsx + c0, *rsx = sm.rsx + c0;
+#define W4A8_EPI(F, B, R) epi_chunk_any<F, B, R, SH>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx)
+                switch (epi_mode) {
+                    case 0: W4A8_EPI(EPI_F32, false, false); break;
+                    case 1: W4A8_EPI(EPI_F32, false, true); break;
+                    case 2: W4A8_EPI(EPI_F32, true, false); break;
+                    case 3: W4A8_EPI(EPI_F32, true, true); break;
+                    case 4: W4A8_EPI(EPI_BF16, false, false); break;
+                    case 5: W4A8_EPI(EPI_BF16, false, true); break;
+                    case 6: W4A8_EPI(EPI_BF16, true, false); break;
+                    case 7: W4A8_EPI(EPI_BF16, true, true); break;
+                    default: W4A8_EPI(EPI_S32, false, false); break;
                 }
+#undef W4A8_EPI
             }
             ptx::tc_fence_before();
             __syncwarp();

@@ -27,16 +27,17 @@ k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (n >= N) return;
     const uint8_t *wr = Wp + (size_t)n * ldp;
-    const float swn = __ldg(sw + n);
+    const float swn = ld_dep(sw + n);
     for (int m = blockIdx.y; m < M; m += gridDim.y) {
         const int8_t *xr = Xq + (size_t)m * ldq;
         int32_t acc = 0;
-        for (int k = 0; k < K; ++k) {
-            const uint32_t b = __ldg(wr + (k >> 1));
-            const int v = (k & 1) ? (int)(b >> 4) : (int)(b & 0xFu);
-            acc += (int32_t)__ldg(xr + k) * ((v ^ 8) - 8);
+        for (int k = 0; k < K; k += 2) {
+            // byte k/2: code k in the low nibble, code k + 1 in the high one
+            const uint32_t b = ld_dep_u8(wr + (k >> 1));
+            acc += ld_dep_s8(xr + k) * ((int)((b & 0xFu) ^ 8u) - 8);
+            if (k + 1 < K) acc += ld_dep_s8(xr + k + 1) * ((int)((b >> 4) ^ 8u) - 8);
         }
-        store_out(Y, ldy, m, n, acc, __ldg(sx + m), swn, bias, flags);
+        store_out(Y, ldy, m, n, acc, ld_dep(sx + m), swn, bias, flags);
     }
 }
 
@@ -58,10 +59,12 @@ k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
 // B fragment of the same thread covers the same slots, so it takes the even
 // and odd bytes of xq[token][128c + 32t + 8j .. +7].
 //
-// PDL: before griddepcontrol.wait the block only asks for its 16 weight rows
-// to be brought into L2 (one bulk prefetch), so the HBM stream starts while
-// the activation-quantization kernel still runs, and every value the kernel
-// computes with is loaded after the wait.
+// PDL: when launched by w4a8_linear behind its activation pass (EARLY), the
+// first batch of weight loads is issued before griddepcontrol.wait, because
+// the activation pass lets this launch start only after all earlier work has
+// completed. Otherwise (w4a8_linear_q, whose predecessor is unknown) the block
+// only asks for its 16 weight rows to be brought into L2 before the wait, and
+// every value it computes with is loaded after it.
 // ---------------------------------------------------------------------------
 constexpr int DEC_WARPS = 8;
 // chunks per warp per batch of loads: 4 for one token group, 2 for two (the
@@ -78,7 +81,7 @@ __device__ __forceinline__ void mma_s8_16832(int32_t (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int NTG>
+template <int NTG, bool EARLY>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
 k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
                 const float *__restrict__ sx,
@@ -88,7 +91,7 @@ k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
     constexpr int DEC_UNROLL = dec_unroll<NTG>();
     static_assert(16 * TOK <= DEC_WARPS * 32, "one epilogue element per thread");
     __shared__ int32_t red[DEC_WARPS][16][TOK + 1];
-    griddep_launch_dependents();  // see k_act_quant: dependents only prefetch weights
+    griddep_launch_dependents();  // dependents only warm L2 before their wait
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -96,11 +99,37 @@ k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
     const int m0 = blockIdx.y * TOK;
     const int nchunks = (ldp + 63) / 64;  // 128-k chunks covering the packed rows
 
-    if (threadIdx.x == 0) {
+    const bool row_lo_ok = n0 + g < N, row_hi_ok = n0 + g + 8 < N;
+    const uint8_t *wlo = Wp + (size_t)(row_lo_ok ? n0 + g : 0) * ldp + 16 * t;
+    const uint8_t *whi = Wp + (size_t)(row_hi_ok ? n0 + g + 8 : 0) * ldp + 16 * t;
+    uint4 wa[DEC_UNROLL], wb[DEC_UNROLL];
+    // One batch of weight loads: chunks cb, cb + DEC_WARPS, ... of this warp.
+    auto load_batch = [&](int cb) {
+#pragma unroll
+        for (int u = 0; u < DEC_UNROLL; ++u) {
+            const int c = cb + u * DEC_WARPS;
+            const int off = 64 * c;  // this thread's piece: off + 16t
+            const bool in = c < nchunks && off + 16 * t < ldp;
+            const uint4 *pa = reinterpret_cast<const uint4 *>(wlo + off);
+            const uint4 *pb = reinterpret_cast<const uint4 *>(whi + off);
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            wa[u] = (in && row_lo_ok) ? ld_dep_cg_v4(pa) : z;
+            wb[u] = (in && row_hi_ok) ? ld_dep_cg_v4(pb) : z;
+        }
+    };
+    if constexpr (EARLY) {
+        // Launched by w4a8_linear right behind its activation pass, which
+        // triggers this launch only after everything enqueued before it has
+        // completed: the weights are final, so they stream now, overlapping
+        // the activation pass, read through L2 (the point of coherence).
+        load_batch(warp);
+    } else if (threadIdx.x == 0) {
+        // The previous kernel may still be writing anything: only warm L2.
         const int rows = min(16, N - n0);
         prefetch_l2_bulk(Wp + (size_t)n0 * ldp, (uint32_t)(rows * ldp));
     }
     griddep_wait();
+    if constexpr (!EARLY) load_batch(warp);
 
     // Epilogue operands, fetched now so their latency hides under the stream:
     // thread e finishes output (channel n0 + e % 16, token m0 + e / 16).
@@ -108,29 +137,23 @@ k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
     const bool e_ok = threadIdx.x < 16 * TOK && n0 + e_ch < N && m0 + e_tk < M;
     float e_sw = 1.0f, e_sx = 1.0f;
     if (e_ok) {
-        e_sw = __ldg(sw + n0 + e_ch);
-        e_sx = __ldg(sx + m0 + e_tk);
+        e_sw = ld_dep(sw + n0 + e_ch);
+        e_sx = ld_dep(sx + m0 + e_tk);
     }
-
-    const bool row_lo_ok = n0 + g < N, row_hi_ok = n0 + g + 8 < N;
-    const uint8_t *wlo = Wp + (size_t)(row_lo_ok ? n0 + g : 0) * ldp + 16 * t;
-    const uint8_t *whi = Wp + (size_t)(row_hi_ok ? n0 + g + 8 : 0) * ldp + 16 * t;
 
     int32_t acc[NTG][4];
 #pragma unroll
     for (int i = 0; i < NTG; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0;
 
     for (int cb = warp; cb < nchunks; cb += DEC_WARPS * DEC_UNROLL) {
-        // Issue every load of this batch before any use: weights and the
-        // matching INT8 activations (an out-of-range piece reads as zeros).
-        uint4 wa[DEC_UNROLL], wb[DEC_UNROLL], xv[DEC_UNROLL][NTG][2];
+        // Issue every load of this batch before any use: weights (the first
+        // batch is already out) and the matching INT8 activations (an
+        // out-of-range piece reads as zeros).
+        if (cb != warp) load_batch(cb);
+        uint4 xv[DEC_UNROLL][NTG][2];
 #pragma unroll
         for (int u = 0; u < DEC_UNROLL; ++u) {
             const int c = cb + u * DEC_WARPS;
-            const int off = 64 * c;                // this thread's piece: off + 16t
-            const bool in = c < nchunks && off + 16 * t < ldp;
-            wa[u] = (in && row_lo_ok) ? __ldg(reinterpret_cast<const uint4 *>(wlo + off)) : make_uint4(0, 0, 0, 0);
-            wb[u] = (in && row_hi_ok) ? __ldg(reinterpret_cast<const uint4 *>(whi + off)) : make_uint4(0, 0, 0, 0);
             const int kbase = 128 * c + 32 * t;
 #pragma unroll
             for (int i = 0; i < NTG; ++i) {
@@ -139,7 +162,7 @@ k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const bool ok = c < nchunks && m < M && kbase + 16 * h < ldq;
-                    xv[u][i][h] = ok ? __ldg(reinterpret_cast<const uint4 *>(xr + 16 * h)) : make_uint4(0, 0, 0, 0);
+                    xv[u][i][h] = ok ? ld_dep_v4(xr + 16 * h) : make_uint4(0, 0, 0, 0);
                 }
             }
         }

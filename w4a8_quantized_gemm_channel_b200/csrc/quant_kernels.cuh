@@ -5,6 +5,10 @@
 //   q = clamp(rne(W[k][n] * sw[n]), -8, 7), packed two per byte along K.
 // Activations (step 3): sx[m] = 127 / max_k |X[m][k]| (1 for an all-zero row);
 //   xq = clamp(rne(X[m][k] * sx[m]), -127, 127).
+// The weight kernels are launched without a programmatic dependency: each
+// starts after all earlier work has finished, so its inputs stay constant
+// while it runs and are read on the read-only path. The activation kernel is
+// a programmatic dependent and reads X with the ld_dep loads.
 #pragma once
 
 #include "common.cuh"
@@ -165,7 +169,7 @@ __global__ void k_weight_scale_finalize(float *__restrict__ sw, int N) {
 // used for the INT8 activations w4a8_linear keeps in its workspace.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float row_load(const float *__restrict__ x, int k, int K) {
-    return k < K ? __ldg(x + k) : 0.0f;
+    return k < K ? ld_dep(x + k) : 0.0f;
 }
 
 template <int U>
@@ -174,7 +178,7 @@ __device__ __forceinline__ void load_unit(const float *__restrict__ x, int k, in
     for (int h = 0; h < U / 4; ++h) {
         const int kk = k + 4 * h;
         if (vec4 && kk + 3 < K) {
-            const float4 f = __ldg(reinterpret_cast<const float4 *>(x + kk));
+            const float4 f = ld_dep_f4(x + kk);
             v[4 * h] = f.x; v[4 * h + 1] = f.y; v[4 * h + 2] = f.z; v[4 * h + 3] = f.w;
         } else {
 #pragma unroll
@@ -215,12 +219,14 @@ k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
     constexpr int G = VPT / U;       // units a thread keeps in registers
     static_assert(THREADS % 32 == 0 && THREADS <= 1024 && VPT % U == 0, "block shape");
     __shared__ float red[THREADS / 32];
-    // Let the next kernel launch now: it only prefetches weights before its
-    // own griddepcontrol.wait, which returns after this grid has finished.
-    // Every block triggers at entry, so all of this grid is resident before
-    // any dependent block can take an SM slot.
+    // X may be written by the previous kernel: wait for it. Only then let the
+    // next kernel launch, so everything enqueued before this kernel has
+    // completed when a dependent starts; the decode kernel relies on that to
+    // stream its weights before its own griddepcontrol.wait (which returns
+    // when this grid has finished). Every block triggers, so all of this grid
+    // is resident before a dependent block can take an SM slot.
+    griddep_wait();
     griddep_launch_dependents();
-    griddep_wait();  // X may be written by the previous kernel
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool in_regs = K <= THREADS * VPT;
     const int units = ldq / U;  // ldq is a multiple of 16
@@ -237,7 +243,7 @@ k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
                 for (int b = 0; b < U; ++b) amax = fmaxf(amax, fabsf(v[i][b]));
             }
         } else {
-            for (int k = threadIdx.x; k < K; k += THREADS) amax = fmaxf(amax, fabsf(__ldg(x + k)));
+            for (int k = threadIdx.x; k < K; k += THREADS) amax = fmaxf(amax, fabsf(ld_dep(x + k)));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));

@@ -119,10 +119,12 @@ unsigned choose_path(int M, int K, int N, unsigned flags) {
 }
 
 // act_perm: Xq uses the k-permuted layout (only the tensor-core path reads it).
+// after_act_pass: the launch directly follows this library's activation pass,
+// so the decode kernel may stream its weights before its dependency wait.
 w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx,
                         const uint8_t *Wp, int ldp, const float *sw, int N,
                         const float *bias, unsigned flags, void *Y, int ldy,
-                        cudaStream_t stream, bool act_perm = false) {
+                        cudaStream_t stream, bool act_perm = false, bool after_act_pass = false) {
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
     const unsigned path = choose_path(M, K, N, flags);
@@ -137,12 +139,10 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
         const int tiles = (M + tok - 1) / tok;
         if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
         dim3 grid((N + 15) / 16, tiles);
-        if (tok == 8)
-            e = launch_pdl(k_linear_decode<1>, grid, dim3(DEC_WARPS * 32), 0, stream,
-                           Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
-        else
-            e = launch_pdl(k_linear_decode<2>, grid, dim3(DEC_WARPS * 32), 0, stream,
-                           Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+        auto kern = tok == 8 ? (after_act_pass ? k_linear_decode<1, true> : k_linear_decode<1, false>)
+                             : (after_act_pass ? k_linear_decode<2, true> : k_linear_decode<2, false>);
+        e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream,
+                       Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
     } else if (path == W4A8_PATH_TC) {
         if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
         w4a8_status st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
@@ -259,7 +259,7 @@ static w4a8_status linear_from_f32(const float *X, int M, int K, int ldx, const 
     const bool perm = path == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
     w4a8_status st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s, perm);
     if (st != W4A8_OK) return st;
-    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s, perm);
+    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s, perm, true);
 }
 
 w4a8_status a8_quantize_rows(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
