@@ -68,6 +68,13 @@ enum {
 #define W4A8_OUT_BF16      0x02u /* Y is bfloat16 [M][ldy], rounded to nearest even */
 #define W4A8_OUT_S32       0x04u /* Y is the raw INT32 accumulator [M][ldy]; no bias, no ReLU */
 #define W4A8_OUT_MASK      0x06u
+/* The caller guarantees that Wp, sw and bias hold their final values and that
+ * no work still pending on the stream writes them (for example: the weights
+ * were quantized when the layer was loaded and the stream has synchronized
+ * since). The kernels may then read them before the previous kernel on the
+ * stream has finished, overlapping the weight stream with its tail. Without
+ * the flag they are read after it; the result is the same either way. */
+#define W4A8_STATIC_WEIGHTS 0x08u
 /* Kernel selection. AUTO picks by shape; the others force one kernel (tests). */
 #define W4A8_PATH_AUTO     0x00u
 #define W4A8_PATH_GENERIC  0x10u /* CUDA-core kernel, any shape */
@@ -123,7 +130,7 @@ W4A8_API w4a8_status a8_quantize_rows(const float *X, int M, int K, int ldx,
  *   X     [M][ldx] float32, ldx >= K.
  *   Wp,sw as produced by w4_quantize_pack for this K and N (pad nibbles 0).
  *   bias  [N] float32 or NULL.
- *   flags W4A8_RELU | one W4A8_OUT_* | one W4A8_PATH_*.
+ *   flags W4A8_RELU | one W4A8_OUT_* | W4A8_STATIC_WEIGHTS | one W4A8_PATH_*.
  *   Y     [M][ldy] out in the W4A8_OUT_* format, ldy >= N.
  *   workspace: device memory of at least w4a8_workspace_size(M, K) bytes,
  *       16-byte aligned; it holds the INT8 activations between kernels and

@@ -342,3 +342,70 @@ def test_decode_linear_matches_quantize_then_linear_q(nat, m, k, n, pad):
     a, c = host(y1), host(y2)
     assert np.array_equal(a.view(np.uint32), c.view(np.uint32))
     assert_f32_close(a, oracle.linear(x, wp, sw, k, bias=b), b)
+
+
+# ------------------------------------- decode with fused quantization ---
+
+@pytest.mark.parametrize("m", [1, 2, 3, 4])
+@pytest.mark.parametrize("k,pad", [(1, 0), (7, 1), (129, 0), (4100, 0), (4100, 3)])
+def test_fused_decode_bit_exact(nat, m, k, pad):
+    """Few-row decode quantizes X inside the product kernel: the INT32
+    accumulators must be the oracle's bit for bit (a zero row included), the
+    float outputs within the layer tolerance, with and without the
+    static-weights promise. `pad` rules out float4 loads of X."""
+    n = 40
+    x, w, b = _case(m, k, n, seed=1100 + 7 * m + k)
+    if m > 1:
+        x[1] = 0.0
+    xbuf = np.zeros((m, k + pad), np.float32)
+    xbuf[:, :k] = x
+    xd = dev(xbuf)[:, :k]
+    wp, sw = oracle.w4_quantize_pack(w)
+    wpd, swd, bd = dev(wp), dev(sw), dev(b)
+    acc_ref = oracle.linear(x, wp, sw, k, out="s32")
+    for static in (False, True):
+        acc = nat.w4a8_linear(xd, wpd, swd, out="s32", path="decode", static_weights=static)
+        assert nat.last_path() == "decode"
+        assert np.array_equal(host(acc), acc_ref)
+        y = nat.w4a8_linear(xd, wpd, swd, bias=bd, relu=True, path="decode", static_weights=static)
+        assert_f32_close(host(y), oracle.linear(x, wp, sw, k, bias=b, relu=True), b)
+        yb = nat.w4a8_linear(xd, wpd, swd, bias=bd, out="bf16", path="decode", static_weights=static)
+        assert_bf16_within_ulp(host(yb.view(torch.int16)),
+                               oracle.linear(x, wp, sw, k, bias=b, out="bf16"))
+
+
+@pytest.mark.parametrize("m,k", [(1, 8192), (1, 8193), (2, 4096), (2, 4097), (4, 2048), (4, 2049),
+                                 (1, 65536), (1, 65537), (2, 32768), (2, 32769), (4, 16384), (4, 16385),
+                                 (8, 8192), (8, 8193)])
+def test_decode_at_kernel_boundaries(nat, m, k):
+    """Both sides of every K at which the few-row decode changes kernels: the
+    activation quantization still fits the product kernel's registers; one
+    weight stage and the INT8 rows still fit a block's shared memory. The
+    result must not depend on the side, with or without the static-weights
+    promise."""
+    n = 24
+    x, w, _ = _case(m, k, n, seed=1200 + m)
+    wp, sw = oracle.w4_quantize_pack(w)
+    ref = oracle.linear(x, wp, sw, k, out="s32")
+    for static in (False, True):
+        acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32", path="decode", static_weights=static)
+        assert np.array_equal(host(acc), ref)
+
+
+@pytest.mark.parametrize("m", [1, 4, 16, 300])
+def test_static_weights_promise_gives_same_bits(nat, m):
+    """W4A8_STATIC_WEIGHTS only lets kernels read the weights earlier: the
+    outputs of w4a8_linear and w4a8_linear_q are the same bits either way."""
+    k, n = 1024, 520
+    x, w, b = _case(m, k, n, seed=1300 + m)
+    wpd, swd = nat.w4_quantize_pack(dev(w))
+    xd, bd = dev(x), dev(b)
+    torch.cuda.synchronize()                 # the weights are settled from here on
+    y0 = host(nat.w4a8_linear(xd, wpd, swd, bias=bd))
+    y1 = host(nat.w4a8_linear(xd, wpd, swd, bias=bd, static_weights=True))
+    assert np.array_equal(y0.view(np.uint32), y1.view(np.uint32))
+    xq, sx = nat.a8_quantize_rows(xd)
+    q0 = host(nat.w4a8_linear_q(xq, sx, k, wpd, swd, bias=bd))
+    q1 = host(nat.w4a8_linear_q(xq, sx, k, wpd, swd, bias=bd, static_weights=True))
+    assert np.array_equal(q0.view(np.uint32), q1.view(np.uint32))
+    assert np.array_equal(y0.view(np.uint32), q0.view(np.uint32))

@@ -77,6 +77,25 @@ __device__ __forceinline__ uint4 ld_dep_cg_v4(const void *p) {
     return v;
 }
 
+// Streaming load (evict-first in L1 and L2) for bytes read once per call.
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Activation quantization (step 3 of "How it works"): the row scale from the
+// row's abs-max (1 for an all-zero row), and one code as a byte.
+__device__ __forceinline__ float act_scale_from_amax(float a) {
+    return a == 0.0f ? 1.0f : __fdiv_rn(127.0f, a);
+}
+__device__ __forceinline__ uint32_t act_code8(float v, float s, bool in) {
+    const int q = in ? min(max(__float2int_rn(__fmul_rn(v, s)), -127), 127) : 0;
+    return (uint32_t)(q & 0xFF);
+}
+
 // Warm L2 with [p, p + bytes) (bytes a multiple of 16, p 16-byte aligned)
 // without returning data: safe to issue before griddepcontrol.wait, because
 // L2 is the point of coherence and no stale value reaches a register.
@@ -100,30 +119,37 @@ __device__ __forceinline__ void unpack_s4x8(uint32_t p, uint32_t &lo, uint32_t &
 // Dequantize one INT32 accumulator and apply the Dense epilogue, in the same
 // float32 operations and order as the method's statement:
 //   y = float(acc) / (sx * sw); y += bias; y = y > 0 ? y : +0.
-__device__ __forceinline__ float dequant_one(int32_t acc, float sxm, float swn,
-                                             const float *__restrict__ bias, int n,
-                                             bool relu) {
+__device__ __forceinline__ float dequant_value(int32_t acc, float sxm, float swn, bool has_bias, float b,
+                                               bool relu) {
     float d = __fmul_rn(sxm, swn);
     float y = __fdiv_rn(__int2float_rn(acc), d);
-    if (bias) y = __fadd_rn(y, ld_dep(bias + n));
+    if (has_bias) y = __fadd_rn(y, b);
     if (relu) y = y > 0.0f ? y : 0.0f;
     return y;
 }
 
-__device__ __forceinline__ void store_out(void *__restrict__ Y, int ldy, int m, int n,
-                                          int32_t acc, float sxm, float swn,
-                                          const float *__restrict__ bias, unsigned flags) {
+// Write output (m, n) in the format `flags` selects; b is bias[n] when a
+// bias is given.
+__device__ __forceinline__ void store_value(void *__restrict__ Y, int ldy, int m, int n, int32_t acc, float sxm,
+                                            float swn, bool has_bias, float b, unsigned flags) {
     size_t off = (size_t)m * (size_t)ldy + (size_t)n;
     unsigned fmt = flags & W4A8_OUT_MASK;
     if (fmt == W4A8_OUT_S32) {
         static_cast<int32_t *>(Y)[off] = acc;
         return;
     }
-    float y = dequant_one(acc, sxm, swn, bias, n, (flags & W4A8_RELU) != 0);
+    float y = dequant_value(acc, sxm, swn, has_bias, b, (flags & W4A8_RELU) != 0);
     if (fmt == W4A8_OUT_BF16)
         static_cast<__nv_bfloat16 *>(Y)[off] = __float2bfloat16_rn(y);
     else
         static_cast<float *>(Y)[off] = y;
+}
+
+__device__ __forceinline__ void store_out(void *__restrict__ Y, int ldy, int m, int n,
+                                          int32_t acc, float sxm, float swn,
+                                          const float *__restrict__ bias, unsigned flags) {
+    const bool has_bias = bias != nullptr && (flags & W4A8_OUT_MASK) != W4A8_OUT_S32;
+    store_value(Y, ldy, m, n, acc, sxm, swn, has_bias, has_bias ? ld_dep(bias + n) : 0.0f, flags);
 }
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return min(max(v, lo), hi); }

@@ -437,18 +437,25 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // A 2-D byte tensor [rows][inner] with the given row stride; tiles of
 // box_inner bytes x box_rows rows; out-of-range elements read as zero.
-inline bool make_map_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows, uint64_t stride,
-                        uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+// 2-D tensor map: `inner` elements of `dtype` per row, `rows` rows `stride`
+// bytes apart; boxes of box_inner x box_rows; reads outside are zero-filled.
+inline bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t inner,
+                        uint64_t rows, uint64_t stride, uint32_t box_inner, uint32_t box_rows,
+                        CUtensorMapSwizzle swz) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {stride};
     cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+    CUresult r = fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+inline bool make_map_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows, uint64_t stride,
+                        uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, rows, stride, box_inner, box_rows, swz);
 }
 
 template <int BT>

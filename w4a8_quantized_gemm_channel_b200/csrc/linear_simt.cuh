@@ -42,7 +42,7 @@ k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
 }
 
 // ---------------------------------------------------------------------------
-// Decode kernel.
+// Decode kernels.
 //
 // Block = 8 warps = one 16-channel row block of the weight matrix; warp w owns
 // the 128-k chunks c = w, w+8, w+16, ... of K, so the block's warps read 512
@@ -59,18 +59,24 @@ k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
 // B fragment of the same thread covers the same slots, so it takes the even
 // and odd bytes of xq[token][128c + 32t + 8j .. +7].
 //
-// PDL: when launched by w4a8_linear behind its activation pass (EARLY), the
-// first batch of weight loads is issued before griddepcontrol.wait, because
-// the activation pass lets this launch start only after all earlier work has
-// completed. Otherwise (w4a8_linear_q, whose predecessor is unknown) the block
-// only asks for its 16 weight rows to be brought into L2 before the wait, and
-// every value it computes with is loaded after it.
+// Only the first kp = round_up(ceil(K/2), 16) bytes of a packed row are read
+// (codes and zero pad nibbles); any row stride past them is never touched.
+//
+// Programmatic dependent launch. Weights are streamed before
+// griddepcontrol.wait only where they are known to be final: behind this
+// library's activation pass (which lets a dependent start only after all
+// earlier work has completed), or when the caller passes
+// W4A8_STATIC_WEIGHTS. Otherwise the block only asks for its weight rows to be
+// brought into L2 before the wait, and loads them after it.
 // ---------------------------------------------------------------------------
 constexpr int DEC_WARPS = 8;
 // chunks per warp per batch of loads: 4 for one token group, 2 for two (the
 // activation fragments double), which keeps two blocks per SM
 template <int NTG>
 constexpr int dec_unroll() { return NTG == 1 ? 4 : 2; }
+
+// Packed bytes of a row that the kernels read: codes plus pad, 16-aligned.
+__host__ __device__ __forceinline__ int packed_row_bytes(int K) { return ((K + 1) / 2 + 15) / 16 * 16; }
 
 __device__ __forceinline__ void mma_s8_16832(int32_t (&c)[4], uint32_t a0, uint32_t a1,
                                              uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -81,55 +87,114 @@ __device__ __forceinline__ void mma_s8_16832(int32_t (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The weight rows n0 + g and n0 + g + 8 as thread (g, t) of a decode warp
+// reads them: one 16-byte piece of each per chunk. Weights are read once per
+// call, so the loads are marked streaming (evict-first), which keeps the
+// activations and outputs in L2.
+template <int UNROLL>
+struct DecodeWeights {
+    const uint8_t *lo, *hi;
+    bool lo_ok, hi_ok;
+    int kp, t16;
+    __device__ __forceinline__ DecodeWeights(const uint8_t *Wp, int ldp, int N, int n0, int g, int t, int K) {
+        lo_ok = n0 + g < N;
+        hi_ok = n0 + g + 8 < N;
+        t16 = 16 * t;
+        lo = Wp + (size_t)(lo_ok ? n0 + g : 0) * ldp + t16;
+        hi = Wp + (size_t)(hi_ok ? n0 + g + 8 : 0) * ldp + t16;
+        kp = packed_row_bytes(K);
+    }
+    // chunks cb, cb + DEC_WARPS, ... (pieces past kp read as zeros)
+    __device__ __forceinline__ void load(int cb, uint4 (&wa)[UNROLL], uint4 (&wb)[UNROLL]) const {
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int off = 64 * (cb + u * DEC_WARPS);
+            const bool in = off + t16 < kp;
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            wa[u] = (in && lo_ok) ? ld_stream_v4(lo + off) : z;
+            wb[u] = (in && hi_ok) ? ld_stream_v4(hi + off) : z;
+        }
+    }
+};
+
+// MMAs of one batch: chunks cb + u * DEC_WARPS (u < UNROLL) that exist.
+template <int NTG, int UNROLL>
+__device__ __forceinline__ void decode_mma_batch(int32_t (&acc)[NTG][4], const uint4 (&wa)[UNROLL],
+                                                 const uint4 (&wb)[UNROLL], const uint4 (&xv)[UNROLL][NTG][2],
+                                                 int cb, int nchunks) {
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+        if (cb + u * DEC_WARPS >= nchunks) continue;  // warp-uniform
+        const uint32_t pa[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
+        const uint32_t pb[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t alo, ahi, blo, bhi;
+            unpack_s4x8(pa[j], alo, ahi);
+            unpack_s4x8(pb[j], blo, bhi);
+#pragma unroll
+            for (int i = 0; i < NTG; ++i) {
+                const uint4 &v = xv[u][i][j >> 1];
+                const uint32_t x0 = (j & 1) ? v.z : v.x;
+                const uint32_t x1 = (j & 1) ? v.w : v.y;
+                const uint32_t b0 = __byte_perm(x0, x1, 0x6420);  // even k
+                const uint32_t b1 = __byte_perm(x0, x1, 0x7531);  // odd k
+                mma_s8_16832(acc[i], alo, blo, ahi, bhi, b0, b1);
+            }
+        }
+    }
+}
+
+// Sum the warps' C fragments (rows g, g+8 = channels, columns 2t, 2t+1 =
+// tokens) through shared memory; returns the block total of output e
+// (channel e % 16, token e / 16) for e < 16 * TOK.
+template <int NTG>
+__device__ __forceinline__ int32_t decode_reduce(int32_t (*red)[16][8 * NTG + 1], const int32_t (&acc)[NTG][4],
+                                                 int warp, int g, int t) {
+#pragma unroll
+    for (int i = 0; i < NTG; ++i) {
+        red[warp][g][8 * i + 2 * t] = acc[i][0];
+        red[warp][g][8 * i + 2 * t + 1] = acc[i][1];
+        red[warp][g + 8][8 * i + 2 * t] = acc[i][2];
+        red[warp][g + 8][8 * i + 2 * t + 1] = acc[i][3];
+    }
+    __syncthreads();
+    int32_t s = 0;
+    if (threadIdx.x < 16 * 8 * NTG) {
+        const int e_ch = threadIdx.x % 16, e_tk = threadIdx.x / 16;
+#pragma unroll
+        for (int w = 0; w < DEC_WARPS; ++w) s += red[w][e_ch][e_tk];
+    }
+    return s;
+}
+
+// Decode kernel on INT8 activations (from the activation pass or the caller).
+// EARLY: the weights are final when the kernel starts (see above).
 template <int NTG, bool EARLY>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
-k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
-                const float *__restrict__ sx,
-                const uint8_t *__restrict__ Wp, int ldp, const float *__restrict__ sw, int N,
-                const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+k_linear_decode(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                const uint8_t *Wp, int ldp, const float *sw, int N,
+                const float *bias, unsigned flags, void *Y, int ldy) {
     constexpr int TOK = 8 * NTG;
-    constexpr int DEC_UNROLL = dec_unroll<NTG>();
+    constexpr int UNROLL = dec_unroll<NTG>();
     static_assert(16 * TOK <= DEC_WARPS * 32, "one epilogue element per thread");
     __shared__ int32_t red[DEC_WARPS][16][TOK + 1];
-    griddep_launch_dependents();  // dependents only warm L2 before their wait
+    griddep_launch_dependents();
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int n0 = blockIdx.x * 16;
     const int m0 = blockIdx.y * TOK;
-    const int nchunks = (ldp + 63) / 64;  // 128-k chunks covering the packed rows
-
-    const bool row_lo_ok = n0 + g < N, row_hi_ok = n0 + g + 8 < N;
-    const uint8_t *wlo = Wp + (size_t)(row_lo_ok ? n0 + g : 0) * ldp + 16 * t;
-    const uint8_t *whi = Wp + (size_t)(row_hi_ok ? n0 + g + 8 : 0) * ldp + 16 * t;
-    uint4 wa[DEC_UNROLL], wb[DEC_UNROLL];
-    // One batch of weight loads: chunks cb, cb + DEC_WARPS, ... of this warp.
-    auto load_batch = [&](int cb) {
-#pragma unroll
-        for (int u = 0; u < DEC_UNROLL; ++u) {
-            const int c = cb + u * DEC_WARPS;
-            const int off = 64 * c;  // this thread's piece: off + 16t
-            const bool in = c < nchunks && off + 16 * t < ldp;
-            const uint4 *pa = reinterpret_cast<const uint4 *>(wlo + off);
-            const uint4 *pb = reinterpret_cast<const uint4 *>(whi + off);
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            wa[u] = (in && row_lo_ok) ? ld_dep_cg_v4(pa) : z;
-            wb[u] = (in && row_hi_ok) ? ld_dep_cg_v4(pb) : z;
-        }
-    };
+    const DecodeWeights<UNROLL> W(Wp, ldp, N, n0, g, t, K);
+    const int nchunks = (W.kp + 63) / 64;
+    uint4 wa[UNROLL], wb[UNROLL];
     if constexpr (EARLY) {
-        // Launched by w4a8_linear right behind its activation pass, which
-        // triggers this launch only after everything enqueued before it has
-        // completed: the weights are final, so they stream now, overlapping
-        // the activation pass, read through L2 (the point of coherence).
-        load_batch(warp);
+        W.load(warp, wa, wb);
     } else if (threadIdx.x == 0) {
-        // The previous kernel may still be writing anything: only warm L2.
-        const int rows = min(16, N - n0);
-        prefetch_l2_bulk(Wp + (size_t)n0 * ldp, (uint32_t)(rows * ldp));
+        prefetch_l2_bulk(Wp + (size_t)n0 * ldp, (uint32_t)(min(16, N - n0) * ldp));
     }
     griddep_wait();
-    if constexpr (!EARLY) load_batch(warp);
+    if constexpr (!EARLY) W.load(warp, wa, wb);
 
     // Epilogue operands, fetched now so their latency hides under the stream:
     // thread e finishes output (channel n0 + e % 16, token m0 + e / 16).
@@ -145,65 +210,31 @@ k_linear_decode(const int8_t *__restrict__ Xq, int M, int K, int ldq,
 #pragma unroll
     for (int i = 0; i < NTG; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0;
 
-    for (int cb = warp; cb < nchunks; cb += DEC_WARPS * DEC_UNROLL) {
+    for (int cb = warp; cb < nchunks; cb += DEC_WARPS * UNROLL) {
         // Issue every load of this batch before any use: weights (the first
         // batch is already out) and the matching INT8 activations (an
         // out-of-range piece reads as zeros).
-        if (cb != warp) load_batch(cb);
-        uint4 xv[DEC_UNROLL][NTG][2];
+        if (cb != warp) W.load(cb, wa, wb);
+        uint4 xv[UNROLL][NTG][2];
 #pragma unroll
-        for (int u = 0; u < DEC_UNROLL; ++u) {
-            const int c = cb + u * DEC_WARPS;
-            const int kbase = 128 * c + 32 * t;
+        for (int u = 0; u < UNROLL; ++u) {
+            const int kbase = 128 * (cb + u * DEC_WARPS) + 32 * t;
 #pragma unroll
             for (int i = 0; i < NTG; ++i) {
                 const int m = m0 + 8 * i + g;
                 const int8_t *xr = Xq + (size_t)m * ldq + kbase;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const bool ok = c < nchunks && m < M && kbase + 16 * h < ldq;
+                    const bool ok = m < M && kbase + 16 * h < ldq;
                     xv[u][i][h] = ok ? ld_dep_v4(xr + 16 * h) : make_uint4(0, 0, 0, 0);
                 }
             }
         }
-#pragma unroll
-        for (int u = 0; u < DEC_UNROLL; ++u) {
-            if (cb + u * DEC_WARPS >= nchunks) continue;  // warp-uniform
-            const uint32_t pa[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
-            const uint32_t pb[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint32_t alo, ahi, blo, bhi;
-                unpack_s4x8(pa[j], alo, ahi);
-                unpack_s4x8(pb[j], blo, bhi);
-#pragma unroll
-                for (int i = 0; i < NTG; ++i) {
-                    const uint4 &v = xv[u][i][j >> 1];
-                    const uint32_t x0 = (j & 1) ? v.z : v.x;
-                    const uint32_t x1 = (j & 1) ? v.w : v.y;
-                    const uint32_t b0 = __byte_perm(x0, x1, 0x6420);  // even k
-                    const uint32_t b1 = __byte_perm(x0, x1, 0x7531);  // odd k
-                    mma_s8_16832(acc[i], alo, blo, ahi, bhi, b0, b1);
-                }
-            }
-        }
+        decode_mma_batch<NTG, UNROLL>(acc, wa, wb, xv, cb, nchunks);
     }
 
-    // C fragment: rows g, g+8 (channels), columns 2t, 2t+1 (tokens).
-#pragma unroll
-    for (int i = 0; i < NTG; ++i) {
-        red[warp][g][8 * i + 2 * t] = acc[i][0];
-        red[warp][g][8 * i + 2 * t + 1] = acc[i][1];
-        red[warp][g + 8][8 * i + 2 * t] = acc[i][2];
-        red[warp][g + 8][8 * i + 2 * t + 1] = acc[i][3];
-    }
-    __syncthreads();
-    if (e_ok) {
-        int32_t s = 0;
-#pragma unroll
-        for (int w = 0; w < DEC_WARPS; ++w) s += red[w][e_ch][e_tk];
-        store_out(Y, ldy, m0 + e_tk, n0 + e_ch, s, e_sx, e_sw, bias, flags);
-    }
+    const int32_t s = decode_reduce<NTG>(red, acc, warp, g, t);
+    if (e_ok) store_out(Y, ldy, m0 + e_tk, n0 + e_ch, s, e_sx, e_sw, bias, flags);
 }
 
 }  // namespace w4a8

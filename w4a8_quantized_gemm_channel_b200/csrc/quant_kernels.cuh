@@ -187,25 +187,20 @@ __device__ __forceinline__ void load_unit(const float *__restrict__ x, int k, in
     }
 }
 
-__device__ __forceinline__ uint32_t code8(float v, float s, bool in) {
-    const int q = in ? clampi(__float2int_rn(__fmul_rn(v, s)), -127, 127) : 0;
-    return (uint32_t)(q & 0xFF);
-}
-
 // Quantize one unit of U consecutive k (k0 = first k) and store it.
 template <int U, bool PERM>
 __device__ __forceinline__ void store_unit(int8_t *__restrict__ row, int k0, int K, float s, const float (&v)[U]) {
     if constexpr (!PERM) {
         uint32_t w = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) w |= code8(v[b], s, k0 + b < K) << (8 * b);
+        for (int b = 0; b < 4; ++b) w |= act_code8(v[b], s, k0 + b < K) << (8 * b);
         *reinterpret_cast<uint32_t *>(row + k0) = w;
     } else {
         uint32_t even = 0, odd = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            even |= code8(v[2 * b], s, k0 + 2 * b < K) << (8 * b);
-            odd |= code8(v[2 * b + 1], s, k0 + 2 * b + 1 < K) << (8 * b);
+            even |= act_code8(v[2 * b], s, k0 + 2 * b < K) << (8 * b);
+            odd |= act_code8(v[2 * b + 1], s, k0 + 2 * b + 1 < K) << (8 * b);
         }
         *reinterpret_cast<uint2 *>(row + k0) = make_uint2(even, odd);
     }
@@ -252,7 +247,7 @@ k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
         float a = red[0];
 #pragma unroll
         for (int i = 1; i < THREADS / 32; ++i) a = fmaxf(a, red[i]);
-        const float s = a == 0.0f ? 1.0f : __fdiv_rn(127.0f, a);
+        const float s = act_scale_from_amax(a);
         if (threadIdx.x == 0) sx[m] = s;
         int8_t *row = Xq + (size_t)m * ldq;
         if (in_regs) {

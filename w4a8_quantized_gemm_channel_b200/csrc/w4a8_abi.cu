@@ -3,12 +3,14 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <cstdio>
+#include <map>
 #include <mutex>
 
 #include "w4a8.h"
 #include "common.cuh"
 #include "quant_kernels.cuh"
 #include "linear_simt.cuh"
+#include "decode_bulk.cuh"
 #include "gemm_tc.cuh"
 
 namespace w4a8 {
@@ -102,7 +104,7 @@ w4a8_status check_common(int M, int K, int N, const uint8_t *Wp, int ldp, const 
     if (fmt == W4A8_OUT_S32 && (bias || (flags & W4A8_RELU))) return W4A8_ERR_INVALID_ARG;
     const size_t esz = fmt == W4A8_OUT_BF16 ? 2 : 4;
     if ((reinterpret_cast<uintptr_t>(Y) & (esz - 1)) != 0) return W4A8_ERR_INVALID_ARG;
-    if (flags & ~(W4A8_RELU | W4A8_OUT_MASK | W4A8_PATH_MASK)) return W4A8_ERR_INVALID_ARG;
+    if (flags & ~(W4A8_RELU | W4A8_OUT_MASK | W4A8_STATIC_WEIGHTS | W4A8_PATH_MASK)) return W4A8_ERR_INVALID_ARG;
     return W4A8_OK;
 }
 
@@ -118,9 +120,132 @@ unsigned choose_path(int M, int K, int N, unsigned flags) {
     return W4A8_PATH_DECODE;
 }
 
+// Kernels that take more than the default 48 KB of shared memory need the
+// limit raised once per device.
+bool raise_smem_limit(const void *kern, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, bool> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(kern, dev);
+    if (done.count(key)) return true;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done[key] = true;
+    return true;
+}
+
+// The persistent decode kernel (one block per SM, a TMA ring of weight
+// stages) serves M <= 8 when its ring and the activation rows fit the
+// shared-memory budget.
+struct RingPlan {
+    bool ok = false;
+    int grid = 0, ring_n = 0;
+    size_t smem = 0;
+};
+
+// Grid and ring for a layer. A block needs ring_n stages next to the INT8
+// rows, within dbulk::SMEM_BUDGET. Short layers (at most two groups per SM):
+// one group per block if two launches' blocks still fit an SM (so the next
+// launch overlaps this one), else one block per SM. Long layers: two blocks
+// per SM, each walking many groups.
+RingPlan ring_plan(int M, int K, int N) {
+    RingPlan p;
+    const DeviceInfo &dev = device_info();
+    if (!dev.ok || M < 1 || M > dbulk::TOK || K > dbulk::X16_MAX_K || tc::encode_fn() == nullptr) return p;
+    const dbulk::Geometry geo(K);
+    const long long groups = (N + dbulk::ROWS - 1) / dbulk::ROWS, sms = dev.sm_count;
+    const long long xs = (long long)geo.xs_bytes(M), stage = geo.stage_bytes();
+    const long long fit = ((long long)dbulk::SMEM_BUDGET - xs) / stage;
+    const long long static_smem = (long long)sizeof(dbulk::Smem) + 1024;
+    auto ring_for = [&](long long grid) {
+        const long long items = (groups + grid - 1) / grid * geo.nst;
+        long long r = items < dbulk::MAX_RING ? items : dbulk::MAX_RING;
+        return r < fit ? r : fit;
+    };
+    auto block_smem = [&](long long ring) { return ring * stage + xs + static_smem; };
+    long long grid;
+    if (groups <= 2 * sms) {
+        const long long per_sm = (groups + sms - 1) / sms;
+        grid = 2 * per_sm * block_smem(ring_for(groups)) <= dbulk::SM_SMEM ? groups : (groups < sms ? groups : sms);
+    } else {
+        grid = 2 * sms;
+    }
+    const long long ring = ring_for(grid);
+    if (ring < 1) return p;
+    p.grid = (int)grid;
+    p.ring_n = (int)ring;
+    p.smem = (size_t)(ring * stage + xs);
+    p.ok = true;
+    return p;
+}
+
+template <bool EARLY, bool FUSED, int R, int J8>
+cudaError_t launch_ring_kernel(const RingPlan &plan, const int8_t *Xq, int ldq, const float *sx, const float *X,
+                               int ldx, int vec4, int M, int K, const uint8_t *Wp, int ldp, const float *sw, int N,
+                               const float *bias, unsigned flags, void *Y, int ldy, cudaStream_t s) {
+    const dbulk::Geometry geo(K);
+    // the packed rows as [N][kp / 8] elements of 8 bytes, stride ldp
+    CUtensorMap tm_w;
+    if (!tc::make_map_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT64, Wp, (uint64_t)(geo.kp / 8), (uint64_t)N,
+                         (uint64_t)ldp, (uint32_t)(geo.sb / 8), dbulk::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    auto kern = dbulk::k_decode_ring<EARLY, FUSED, R, J8>;
+    if (!raise_smem_limit(reinterpret_cast<const void *>(kern), dbulk::SMEM_BUDGET)) return cudaErrorInvalidValue;
+    return launch_pdl(kern, dim3(plan.grid), dim3(dbulk::THREADS), plan.smem, s, tm_w, Xq, ldq, sx, X, ldx, vec4, M,
+                      K, sw, N, bias, flags, Y, ldy, plan.ring_n);
+}
+
+// Product on INT8 activations through the persistent decode kernel.
+cudaError_t launch_ring_q(const RingPlan &plan, bool early, const int8_t *Xq, int ldq, const float *sx, int M,
+                          int K, const uint8_t *Wp, int ldp, const float *sw, int N, const float *bias,
+                          unsigned flags, void *Y, int ldy, cudaStream_t s) {
+    if (early)
+        return launch_ring_kernel<true, false, 1, 1>(plan, Xq, ldq, sx, nullptr, 0, 0, M, K, Wp, ldp, sw, N,
+                                                           bias, flags, Y, ldy, s);
+    return launch_ring_kernel<false, false, 1, 1>(plan, Xq, ldq, sx, nullptr, 0, 0, M, K, Wp, ldp, sw, N, bias,
+                                                        flags, Y, ldy, s);
+}
+
+// Decode with the activation quantization fused in: the block keeps R rows
+// x J8 units of 8 floats per thread in registers (R * J8 <= 4), so M <= R and
+// the stages' k <= 2048 J8.
+int fq_rows(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+int fq_j8(int K) {  // units per row and thread to cover the stages' k, rounded up to a power of 2
+    const int j = (dbulk::Geometry(K).pitch - 16 + 2047) / 2048;
+    int p = 1;
+    while (p < j) p *= 2;
+    return p;
+}
+bool fq_eligible(int M, int K, int N, unsigned path) {
+    return path == W4A8_PATH_DECODE && ring_plan(M, K, N).ok && fq_rows(M) * fq_j8(K) <= 4;
+}
+
+w4a8_status launch_fq(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp,
+                      const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                      cudaStream_t s) {
+    const int vec4 = aligned16(X) && (ldx % 4 == 0);
+    const RingPlan plan = ring_plan(M, K, N);
+    const bool early = (flags & W4A8_STATIC_WEIGHTS) != 0;
+    cudaError_t e = cudaErrorInvalidValue;
+#define W4A8_FQ(E, R, J)                                                                                       \
+    if (early == E && fq_rows(M) == R && fq_j8(K) == J)                                                        \
+        e = launch_ring_kernel<E, true, R, J>(plan, nullptr, 0, nullptr, X, ldx, vec4, M, K, Wp, ldp, sw, N, \
+                                                    bias, flags, Y, ldy, s);
+    W4A8_FQ(true, 1, 1) W4A8_FQ(true, 1, 2) W4A8_FQ(true, 1, 4) W4A8_FQ(true, 2, 1) W4A8_FQ(true, 2, 2)
+    W4A8_FQ(true, 4, 1)
+    W4A8_FQ(false, 1, 1) W4A8_FQ(false, 1, 2) W4A8_FQ(false, 1, 4) W4A8_FQ(false, 2, 1) W4A8_FQ(false, 2, 2)
+    W4A8_FQ(false, 4, 1)
+#undef W4A8_FQ
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    t_last_path = W4A8_PATH_DECODE;
+    return W4A8_OK;
+}
+
 // act_perm: Xq uses the k-permuted layout (only the tensor-core path reads it).
 // after_act_pass: the launch directly follows this library's activation pass,
-// so the decode kernel may stream its weights before its dependency wait.
+// so the decode kernel may stream its weights before its dependency wait (as
+// it may when the caller passes W4A8_STATIC_WEIGHTS).
 w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx,
                         const uint8_t *Wp, int ldp, const float *sw, int N,
                         const float *bias, unsigned flags, void *Y, int ldy,
@@ -134,13 +259,17 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
         dim3 grid((N + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
         e = launch_pdl(k_linear_generic, grid, dim3(128), 0, stream,
                        Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+    } else if (path == W4A8_PATH_DECODE && ring_plan(M, K, N).ok) {
+        const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
+        e = launch_ring_q(ring_plan(M, K, N), early, Xq, ldq, sx, M, K, Wp, ldp, sw, N, bias, flags, Y, ldy, stream);
     } else if (path == W4A8_PATH_DECODE) {
         const int tok = M <= 8 ? 8 : 16;
         const int tiles = (M + tok - 1) / tok;
         if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
         dim3 grid((N + 15) / 16, tiles);
-        auto kern = tok == 8 ? (after_act_pass ? k_linear_decode<1, true> : k_linear_decode<1, false>)
-                             : (after_act_pass ? k_linear_decode<2, true> : k_linear_decode<2, false>);
+        const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
+        auto kern = tok == 8 ? (early ? k_linear_decode<1, true> : k_linear_decode<1, false>)
+                             : (early ? k_linear_decode<2, true> : k_linear_decode<2, false>);
         e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream,
                        Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
     } else if (path == W4A8_PATH_TC) {
@@ -251,11 +380,13 @@ static w4a8_status launch_act_quant(const float *X, int M, int K, int ldx, int8_
 }
 
 // Steps 3-6 on float32 activations with the INT8 copy in `ws`: the path is
-// chosen first, so the tensor-core GEMM gets its k-permuted activation layout.
+// chosen first, so the tensor-core GEMM gets its k-permuted activation layout
+// and a few-row decode quantizes inside its own kernel.
 static w4a8_status linear_from_f32(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp,
                                    const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
                                    const Workspace &ws, cudaStream_t s) {
     const unsigned path = choose_path(M, K, N, flags);
+    if (fq_eligible(M, K, N, path)) return launch_fq(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
     const bool perm = path == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
     w4a8_status st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s, perm);
     if (st != W4A8_OK) return st;

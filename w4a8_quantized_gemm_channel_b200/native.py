@@ -19,6 +19,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 
 RELU = 0x01
 OUT_F32, OUT_BF16, OUT_S32 = 0x00, 0x02, 0x04
+STATIC_WEIGHTS = 0x08
 PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TC = 0x00, 0x10, 0x20, 0x30
 MAX_K = 2097152
 
@@ -98,8 +99,9 @@ def workspace_size(m: int, k: int) -> int:
     return lib.w4a8_workspace_size(m, k)
 
 
-def flags_for(relu: bool = False, out: str = "f32", path: str = "auto") -> int:
-    return (RELU if relu else 0) | _OUT[out] | _PATH[path]
+def flags_for(relu: bool = False, out: str = "f32", path: str = "auto",
+              static_weights: bool = False) -> int:
+    return (RELU if relu else 0) | _OUT[out] | _PATH[path] | (STATIC_WEIGHTS if static_weights else 0)
 
 
 def w4_quantize_pack(w: torch.Tensor, wp: torch.Tensor | None = None,
@@ -141,8 +143,12 @@ def _out_tensor(y, m, n, out, device):
 def w4a8_linear(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
                 bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
                 path: str = "auto", y: torch.Tensor | None = None,
-                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Y[M][N] = dequant(quant8(X) @ unpack(Wp)^T) (+bias, ReLU) for X[M][K] float32."""
+                workspace: torch.Tensor | None = None, stream=None,
+                static_weights: bool = False) -> torch.Tensor:
+    """Y[M][N] = dequant(quant8(X) @ unpack(Wp)^T) (+bias, ReLU) for X[M][K] float32.
+
+    static_weights: promise that wp, sw and bias are final and not written by
+    work still pending on the stream (W4A8_STATIC_WEIGHTS)."""
     ldx = _rowmajor(x, "X")
     ldp = _rowmajor(wp, "Wp")
     m, k = x.shape
@@ -152,7 +158,7 @@ def w4a8_linear(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
     _check(lib.w4a8_linear(_ptr(x), m, k, ldx, _ptr(wp), ldp, _ptr(sw), n, _ptr(bias),
-                           flags_for(relu, out, path), _ptr(y), ldy, _ptr(workspace),
+                           flags_for(relu, out, path, static_weights), _ptr(y), ldy, _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)),
            "w4a8_linear")
     return y
@@ -161,7 +167,7 @@ def w4a8_linear(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
 def w4a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor,
                   sw: torch.Tensor, bias: torch.Tensor | None = None, relu: bool = False,
                   out: str = "f32", path: str = "auto", y: torch.Tensor | None = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, static_weights: bool = False) -> torch.Tensor:
     """Y from INT8 activations Xq[M][ldq] (first k bytes of each row) and sx[M]."""
     ldq = _rowmajor(xq, "Xq")
     ldp = _rowmajor(wp, "Wp")
@@ -169,7 +175,7 @@ def w4a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor,
     n = wp.shape[0]
     y, ldy = _out_tensor(y, m, n, out, xq.device)
     _check(lib.w4a8_linear_q(_ptr(xq), m, k, ldq, _ptr(sx), _ptr(wp), ldp, _ptr(sw), n,
-                             _ptr(bias), flags_for(relu, out, path), _ptr(y), ldy,
+                             _ptr(bias), flags_for(relu, out, path, static_weights), _ptr(y), ldy,
                              _stream(stream)),
            "w4a8_linear_q")
     return y
@@ -181,7 +187,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 def w4a8_linear_noalloc(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
                         bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
                         path: str = "auto", y: torch.Tensor | None = None,
-                        stream=None) -> torch.Tensor:
+                        stream=None, static_weights: bool = False) -> torch.Tensor:
     """w4a8_linear without a caller workspace: the INT8 activations live in the
     library's fixed per-device scratch array (see include/w4a8.h)."""
     ldx = _rowmajor(x, "X")
@@ -190,7 +196,8 @@ def w4a8_linear_noalloc(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
     n = wp.shape[0]
     y, ldy = _out_tensor(y, m, n, out, x.device)
     _check(lib.w4a8_linear_noalloc(_ptr(x), m, k, ldx, _ptr(wp), ldp, _ptr(sw), n, _ptr(bias),
-                                   flags_for(relu, out, path), _ptr(y), ldy, _stream(stream)),
+                                   flags_for(relu, out, path, static_weights), _ptr(y), ldy,
+                                   _stream(stream)),
            "w4a8_linear_noalloc")
     return y
 
