@@ -188,6 +188,11 @@ W4A8_API w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx,
  * last successful w4a8_linear / w4a8_linear_q call enqueued; 0 if none. */
 W4A8_API unsigned w4a8_last_path(void);
 
+/* How many kernels the calling thread's last successful w4a8_linear /
+ * w4a8_linear_q / w4a8_linear_noalloc call enqueued (1 or 2; 0 if none, or
+ * if that call had M == 0). */
+W4A8_API unsigned w4a8_last_launch_count(void);
+
 /* Read (and with clear != 0, reset) the current device's status word, which
  * kernels set on an internal fault. Synchronizes `stream` first. */
 W4A8_API w4a8_status w4a8_get_device_status(int clear, void *stream);

@@ -17,6 +17,7 @@ namespace w4a8 {
 namespace {
 
 thread_local unsigned t_last_path = 0;
+thread_local unsigned t_last_launches = 0;
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -239,6 +240,7 @@ w4a8_status launch_fq(const float *X, int M, int K, int ldx, const uint8_t *Wp, 
 #undef W4A8_FQ
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
     t_last_path = W4A8_PATH_DECODE;
+    t_last_launches = 1;
     return W4A8_OK;
 }
 
@@ -282,6 +284,7 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     }
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
     t_last_path = path;
+    t_last_launches = 1;
     return W4A8_OK;
 }
 
@@ -390,7 +393,9 @@ static w4a8_status linear_from_f32(const float *X, int M, int K, int ldx, const 
     const bool perm = path == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
     w4a8_status st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s, perm);
     if (st != W4A8_OK) return st;
-    return run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s, perm, true);
+    st = run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s, perm, true);
+    if (st == W4A8_OK) t_last_launches = 2;
+    return st;
 }
 
 w4a8_status a8_quantize_rows(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
@@ -409,7 +414,7 @@ w4a8_status w4a8_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp
     w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
     if (st != W4A8_OK) return st;
     if (ldx < K) return W4A8_ERR_INVALID_ARG;
-    if (M == 0) return W4A8_OK;
+    if (M == 0) { t_last_launches = 0; return W4A8_OK; }
     if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
     if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
     if (workspace_bytes < w4a8_workspace_size(M, K)) return W4A8_ERR_WORKSPACE;
@@ -425,7 +430,7 @@ w4a8_status w4a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *
     w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
     if (st != W4A8_OK) return st;
     if (ldq < K || ldq % 16 != 0) return W4A8_ERR_INVALID_ARG;
-    if (M == 0) return W4A8_OK;
+    if (M == 0) { t_last_launches = 0; return W4A8_OK; }
     if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
     return run_product(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
                        static_cast<cudaStream_t>(stream));
@@ -437,7 +442,7 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
     w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
     if (st != W4A8_OK) return st;
     if (ldx < K) return W4A8_ERR_INVALID_ARG;
-    if (M == 0) return W4A8_OK;
+    if (M == 0) { t_last_launches = 0; return W4A8_OK; }
     if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
     if (w4a8_workspace_size(M, K) > (size_t)W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
     if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
@@ -449,6 +454,8 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
 }
 
 unsigned w4a8_last_path(void) { return t_last_path; }
+
+unsigned w4a8_last_launch_count(void) { return t_last_launches; }
 
 w4a8_status w4a8_get_device_status(int clear, void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

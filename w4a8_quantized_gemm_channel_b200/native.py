@@ -40,6 +40,7 @@ SIGNATURES = {
     "w4a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_last_path": (_U, []),
+    "w4a8_last_launch_count": (_U, []),
     "w4a8_get_device_status": (_I, [_I, _P]),
     "w4a8_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -204,6 +205,10 @@ def w4a8_linear_noalloc(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
 
 def last_path() -> str:
     return PATH_NAMES.get(lib.w4a8_last_path(), "none")
+
+
+def last_launch_count() -> int:
+    return lib.w4a8_last_launch_count()
 
 
 def get_device_status(clear: bool = False, stream=None) -> int:
