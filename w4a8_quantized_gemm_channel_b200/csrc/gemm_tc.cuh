@@ -16,8 +16,8 @@
 //    and a warp stores 32 consecutive channels of a token row at once.
 //
 // One persistent CTA per SM walks the (channel tile, token tile) grid.
-// Warp roles (12 warps): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues the MMAs, warps 4-7 unpack weights, warps 8-11 run the epilogue.
+// Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs,
+// warps 4-11 (two warpgroups) unpack weights, warps 12-15 run the epilogue.
 // Shared-memory stages and TMEM A slots form a STAGES-deep ring; the
 // accumulator is double-buffered so the epilogue of one tile overlaps the
 // main loop of the next. Every mbarrier wait is bounded (see ptx::mbar_wait).
@@ -34,24 +34,28 @@ namespace w4a8 {
 namespace tc {
 
 constexpr int BM = 128;            // output channels per tile (MMA M)
-constexpr int BK = 128;            // k per stage
+constexpr int BK = 256;            // k per stage (one pipeline iteration)
 constexpr int MMA_K = 32;          // k per kind::i8 instruction
-// Two rings. Shared-memory stages (TMA -> unpack/MMA) are deep, so loads run
-// far ahead of the tensor pipe: 8 x 24 KB = 192 KB, which also keeps a second
-// CTA (that would block in tcgen05.alloc of the whole TMEM) off the SM. TMEM A
-// slots (unpack -> MMA) only cover the short unpack hop: 6 x 32 columns next
-// to the two 128-column accumulators.
-constexpr int STAGES = 8;
-constexpr int A_SLOTS = 6;
+constexpr int XBOX = 128;          // bytes of k per activation TMA box (the 128-byte swizzle span)
+// The MMA thread pays a fixed cost per pipeline iteration (barrier waits, the
+// commit) that does not depend on the MMA shape, so an iteration carries 8
+// MMAs (BK = 256). Two rings. Shared-memory stages (TMA -> unpack/MMA):
+// 4 x 48 KB = 192 KB, which also keeps a second CTA (that would block in
+// tcgen05.alloc of the whole TMEM) off the SM. TMEM A slots (unpack -> MMA)
+// cover the unpack hop: 4 x 64 columns next to the two 128-column
+// accumulators.
+constexpr int STAGES = 4;
+constexpr int A_SLOTS = 4;
 // Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
 // it % UNPACK_WG, so the groups overlap their shared-memory reads, integer
 // work and TMEM stores.
-constexpr int UNPACK_WG = 3;
+constexpr int UNPACK_WG = 2;
 static_assert(A_SLOTS % UNPACK_WG == 0, "each warpgroup owns fixed TMEM slots");
 // The unpack warps reuse A slot it % A_SLOTS once the stage barrier of
 // iteration it - A_SLOTS has flipped; that barrier is not reused before
 // iteration it - A_SLOTS + STAGES >= it, which cannot have run yet.
 static_assert(STAGES >= A_SLOTS, "A-slot reuse waits on a stage barrier");
+static_assert(BK % XBOX == 0 && XBOX % MMA_K == 0, "activation boxes hold whole MMA k steps");
 constexpr int FIRST_UNPACK_WARP = 4;
 constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + 4 * UNPACK_WG;
 constexpr int NUM_THREADS = 32 * (FIRST_EPI_WARP + 4);
@@ -61,8 +65,8 @@ constexpr int W_TILE_BYTES = BM * BK / 2;
 
 template <int BT>
 struct alignas(1024) Smem {
-    uint8_t act[STAGES][BT * BK];        // activation tiles, 128B-swizzled rows
-    uint8_t wpk[STAGES][W_TILE_BYTES];   // packed weight tiles, 64B-swizzled rows
+    uint8_t act[STAGES][BT * BK];        // activation tiles: BK / XBOX boxes of [BT][128 B], 128B-swizzled
+    uint8_t wpk[STAGES][W_TILE_BYTES];   // packed weight tiles [BM][128 B], 128B-swizzled
     uint64_t full[STAGES];               // TMA landed (tx-count barrier)
     uint64_t empty[STAGES];              // MMAs reading the stage finished
     uint64_t aready[A_SLOTS];            // A slot written to TMEM (4 unpack warps)
@@ -200,7 +204,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                     if (!ptx::mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&sm.full[stage], BT * BK + W_TILE_BYTES);
                     ptx::tma_load_2d(sm.wpk[stage], &tm_w, kb * (BK / 2), n_tile * BM, &sm.full[stage]);
-                    ptx::tma_load_2d(sm.act[stage], &tm_x, kb * BK, m_tile * BT, &sm.full[stage]);
+#pragma unroll
+                    for (int h = 0; h < BK / XBOX; ++h)
+                        ptx::tma_load_2d(sm.act[stage] + h * BT * XBOX, &tm_x, kb * BK + h * XBOX, m_tile * BT,
+                                         &sm.full[stage]);
                     issued |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -242,9 +249,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 const uint32_t d = tmem + (uint32_t)d_col<BT>(buf);
                 const uint32_t a = tmem + (uint32_t)a_col<BT>(slot);
                 const uint32_t b = ptx::smem_addr(sm.act[stage]);
+                // k step kk reads the activation box kk / 4 at byte offset 32 (kk % 4)
+                constexpr int KPB = XBOX / MMA_K;
 #pragma unroll
                 for (int kk = 0; kk < KSTEPS - 1; ++kk)
-                    ptx::mma_i8_ts(d, a + kk * (MMA_K / 4), ptx::sdesc_k_sw128(b + kk * MMA_K), idesc,
+                    ptx::mma_i8_ts(d, a + kk * (MMA_K / 4),
+                                   ptx::sdesc_k_sw128(b + (kk / KPB) * BT * XBOX + (kk % KPB) * MMA_K), idesc,
                                    (kb | kk) != 0);
                 // next ring positions; wait for their operands while the MMAs
                 // already queued keep the tensor core busy
@@ -255,7 +265,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 const bool next_ok = it + 1 < total ? (ptx::mbar_wait(&sm.full[nstage], nsphase, abort) &&
                                                        ptx::mbar_wait(&sm.aready[nslot], naphase, abort))
                                                     : true;
-                ptx::mma_i8_ts(d, a + (KSTEPS - 1) * (MMA_K / 4), ptx::sdesc_k_sw128(b + (KSTEPS - 1) * MMA_K),
+                ptx::mma_i8_ts(d, a + (KSTEPS - 1) * (MMA_K / 4),
+                               ptx::sdesc_k_sw128(b + ((KSTEPS - 1) / KPB) * BT * XBOX + ((KSTEPS - 1) % KPB) * MMA_K),
                                idesc, 1u);
                 any = true;
                 ptx::mma_commit(&sm.empty[stage]);
@@ -275,11 +286,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
         }
     } else if (warp >= FIRST_UNPACK_WARP && warp < FIRST_EPI_WARP) {
         // ---------------------------------------------------- weight unpack
-        // Thread r owns output-channel row r of the tile: 64 packed bytes per
-        // stage, read from the 64B-swizzled tile (16-byte chunk c of row r
-        // sits at chunk c ^ ((r >> 1) & 3)), expanded to 128 INT8 in k order
-        // and stored to TMEM lane r, 32 columns. Warpgroup wg takes the
-        // pipeline iterations it with it % UNPACK_WG == wg.
+        // Thread r owns output-channel row r of the tile: 128 packed bytes per
+        // stage, read from the 128B-swizzled tile (16-byte chunk c of row r
+        // sits at chunk c ^ (r & 7)), expanded to 256 INT8 in k order and
+        // stored to TMEM lane r, 64 columns (two stores of 32). Warpgroup wg
+        // takes the pipeline iterations it with it % UNPACK_WG == wg.
         const int q = warp & 3;
         const int wg = (warp - FIRST_UNPACK_WARP) >> 2;
         const int r = q * 32 + lane;
@@ -307,31 +318,34 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint8_t *row = sm.wpk[stage] + r * (BK / 2);
-                const int sx_ = (r >> 1) & 3;
-                uint32_t out[32];
+                const int sx_ = r & 7;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * (c ^ sx_));
-                    const uint32_t p[4] = {v.x, v.y, v.z, v.w};
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t out[32];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t lo, hi;  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
-                        if constexpr (UNPACK == UNPACK_SEXT) {
-                            unpack_s4x8(p[j], lo, hi);
-                        } else {
-                            lo = (p[j] << 4) & 0xF0F0F0F0u;
-                            hi = p[j] & 0xF0F0F0F0u;
-                        }
-                        if constexpr (UNPACK == UNPACK_X16_PERM) {
-                            out[8 * c + 2 * j] = lo;
-                            out[8 * c + 2 * j + 1] = hi;
-                        } else {
-                            out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
-                            out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * ((4 * half + c) ^ sx_));
+                        const uint32_t p[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t lo, hi;  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
+                            if constexpr (UNPACK == UNPACK_SEXT) {
+                                unpack_s4x8(p[j], lo, hi);
+                            } else {
+                                lo = (p[j] << 4) & 0xF0F0F0F0u;
+                                hi = p[j] & 0xF0F0F0F0u;
+                            }
+                            if constexpr (UNPACK == UNPACK_X16_PERM) {
+                                out[8 * c + 2 * j] = lo;
+                                out[8 * c + 2 * j + 1] = hi;
+                            } else {
+                                out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
+                                out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                            }
                         }
                     }
+                    ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)(a_col<BT>(slot) + 32 * half), out);
                 }
-                ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)a_col<BT>(slot), out);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -474,8 +488,8 @@ inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *
     if (attr_err != cudaSuccess) return W4A8_ERR_CUDA;
     CUtensorMap tm_w, tm_x;
     if (!make_map_u8(&tm_w, Wp, (uint64_t)ldp, (uint64_t)N, (uint64_t)ldp, BK / 2, BM,
-                     CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_u8(&tm_x, Xq, (uint64_t)ldq, (uint64_t)M, (uint64_t)ldq, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B))
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_u8(&tm_x, Xq, (uint64_t)ldq, (uint64_t)M, (uint64_t)ldq, XBOX, BT, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     const long long tiles = (long long)((M + BT - 1) / BT) * ((N + BM - 1) / BM);
     const int grid = (int)(tiles < sm_count ? tiles : sm_count);
