@@ -37,15 +37,17 @@ constexpr int BM = 128;            // output channels per tile (MMA M)
 constexpr int BK = 256;            // k per stage (one pipeline iteration)
 constexpr int MMA_K = 32;          // k per kind::i8 instruction
 constexpr int XBOX = 128;          // bytes of k per activation TMA box (the 128-byte swizzle span)
-// The MMA thread pays a fixed cost per pipeline iteration (barrier waits, the
-// commit) that does not depend on the MMA shape, so an iteration carries 8
-// MMAs (BK = 256). Two rings. Shared-memory stages (TMA -> unpack/MMA):
-// 4 x 48 KB = 192 KB, which also keeps a second CTA (that would block in
-// tcgen05.alloc of the whole TMEM) off the SM. TMEM A slots (unpack -> MMA)
-// cover the unpack hop: 4 x 64 columns next to the two 128-column
-// accumulators.
-constexpr int STAGES = 4;
-constexpr int A_SLOTS = 4;
+// The tensor core queues about one MMA ahead of the issuing thread, so every
+// stretch of other work on that thread (barrier waits, the commit, loop
+// bookkeeping) longer than one MMA leaves the pipe idle. Hence wide MMAs (a
+// token tile of BT = 192 gives N = 192, 96 tensor cycles each) and 8 of them
+// per pipeline iteration (BK = 256). Two rings. Shared-memory stages (TMA ->
+// unpack/MMA): 3 x 64 KB = 192 KB, which also keeps a second CTA (that would
+// block in tcgen05.alloc of the whole TMEM) off the SM. TMEM A slots (unpack
+// -> MMA): 2 x 64 columns next to the two 192-column accumulators.
+constexpr int BT_TILE = 192;       // tokens per tile (MMA N)
+constexpr int STAGES = 3;
+constexpr int A_SLOTS = 2;
 // Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
 // it % UNPACK_WG, so the groups overlap their shared-memory reads, integer
 // work and TMEM stores.
@@ -520,13 +522,13 @@ inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const
                                   int ldy, int sm_count, cudaStream_t stream, bool act_perm = false) {
     if (K > tc::TC_X16_MAX_K) {
         if (act_perm) return W4A8_ERR_UNSUPPORTED;
-        return tc::launch<128, tc::UNPACK_SEXT>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
+        return tc::launch<tc::BT_TILE, tc::UNPACK_SEXT>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
                                                 stream);
     }
     if (act_perm)
-        return tc::launch<128, tc::UNPACK_X16_PERM>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+        return tc::launch<tc::BT_TILE, tc::UNPACK_X16_PERM>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
                                                     sm_count, stream);
-    return tc::launch<128, tc::UNPACK_X16>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
+    return tc::launch<tc::BT_TILE, tc::UNPACK_X16>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
                                            stream);
 }
 
