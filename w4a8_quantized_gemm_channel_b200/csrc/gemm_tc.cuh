@@ -223,12 +223,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
         }
     } else if (warp == 1) {
         // ---------------------------------------------------- MMA issuer
-        // One iteration = one stage (BK k) of one tile: 4 MMAs into the tile's
-        // accumulator, then one commit that frees the shared-memory stage (and,
+        // One iteration = one stage (BK k) of one tile: 8 MMAs into the tile's
+        // accumulator and one commit that frees the shared-memory stage (and,
         // A_SLOTS iterations later, the TMEM A slot: the unpack warps wait on the
         // same barrier). The tensor core queues only about one MMA ahead, so the
-        // waits for the next iteration's operands are done before the last MMA
-        // of this one is issued, while the queued MMAs still run.
+        // wait for the next iteration's operands is done before the last MMA
+        // of this one is issued, while the queued MMAs still run. (Committing
+        // behind the next iteration's first MMA instead was measured slower:
+        // with two A slots it delays the unpack of the slot's next use.)
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_i8(BM, BT);
             constexpr int KSTEPS = BK / MMA_K;
@@ -238,10 +240,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             // on this thread, which paces the tensor core)
             int stage = 0, slot = 0, kb = 0, buf = 0;
             uint32_t sphase = 0, aphase = 0, bphase = 0;
-            // the unpack warps signal aready only after their own wait on
-            // full[], so the TMA data of that iteration has landed as well
-            bool ok = total > 0 ? (ptx::mbar_wait(&sm.full[0], 0, abort) && ptx::mbar_wait(&sm.aready[0], 0, abort))
-                                : true;
+            // The unpack warps arrive on aready only after their own wait on
+            // full[] of the same iteration, so once aready has flipped the
+            // TMA data of that iteration has landed as well: the MMA thread
+            // waits on aready alone.
+            bool ok = total > 0 ? ptx::mbar_wait(&sm.aready[0], 0, abort) : true;
             bool any = false;
             for (int it = 0; it < total && ok; ++it) {
                 if (kb == 0) {
@@ -264,9 +267,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 uint32_t nsphase = sphase, naphase = aphase;
                 if (nstage == STAGES) { nstage = 0; nsphase ^= 1u; }
                 if (nslot == A_SLOTS) { nslot = 0; naphase ^= 1u; }
-                const bool next_ok = it + 1 < total ? (ptx::mbar_wait(&sm.full[nstage], nsphase, abort) &&
-                                                       ptx::mbar_wait(&sm.aready[nslot], naphase, abort))
-                                                    : true;
+                const bool next_ok = it + 1 < total ? ptx::mbar_wait(&sm.aready[nslot], naphase, abort) : true;
                 ptx::mma_i8_ts(d, a + (KSTEPS - 1) * (MMA_K / 4),
                                ptx::sdesc_k_sw128(b + ((KSTEPS - 1) / KPB) * BT * XBOX + ((KSTEPS - 1) % KPB) * MMA_K),
                                idesc, 1u);
