@@ -18,7 +18,7 @@
 // One persistent CTA per SM walks the (channel tile, token tile) grid.
 // Warp roles: warp 0 issues TMA loads, warp 1 owns TMEM and issues the MMAs,
 // warps 4-11 (two warpgroups) unpack weights, warps 12-15 run the epilogue.
-// Shared-memory stages and TMEM A slots form a STAGES-deep ring; the
+// Shared-memory stages and TMEM A slots form rings; the
 // accumulator is double-buffered so the epilogue of one tile overlaps the
 // main loop of the next. Every mbarrier wait is bounded (see ptx::mbar_wait).
 #pragma once
@@ -41,22 +41,22 @@ constexpr int XBOX = 128;          // bytes of k per activation TMA box (the 128
 // stretch of other work on that thread (barrier waits, the commit, loop
 // bookkeeping) longer than one MMA leaves the pipe idle. Hence wide MMAs (a
 // token tile of BT = 192 gives N = 192, 96 tensor cycles each) and 8 of them
-// per pipeline iteration (BK = 256). Two rings. Shared-memory stages (TMA ->
-// unpack/MMA): 3 x 64 KB = 192 KB, which also keeps a second CTA (that would
-// block in tcgen05.alloc of the whole TMEM) off the SM. TMEM A slots (unpack
-// -> MMA): 2 x 64 columns next to the two 192-column accumulators.
-constexpr int BT_TILE = 192;       // tokens per tile (MMA N)
-constexpr int STAGES = 3;
-constexpr int A_SLOTS = 2;
+// per pipeline iteration (BK = 256). Smaller token tiles (128, 64) serve
+// layers whose few rows or few tiles would leave a 192-token grid padded or
+// mostly idle; the host picks BT per call.
+//
+// Two rings per token tile. Shared-memory stages (TMA -> unpack/MMA) take
+// 192 KB, which also keeps a second CTA (that would block in tcgen05.alloc
+// of the whole TMEM) off the SM. TMEM A slots (unpack -> MMA) of 64 columns
+// sit next to the two BT-column accumulators.
+template <int BT> struct Ring;
+template <> struct Ring<192> { static constexpr int STAGES = 3, A_SLOTS = 2; };  // 3 x 64 KB, 384 + 128 cols
+template <> struct Ring<128> { static constexpr int STAGES = 4, A_SLOTS = 4; };  // 4 x 48 KB, 256 + 256 cols
+template <> struct Ring<64> { static constexpr int STAGES = 6, A_SLOTS = 4; };   // 6 x 32 KB, 128 + 256 cols
 // Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
 // it % UNPACK_WG, so the groups overlap their shared-memory reads, integer
 // work and TMEM stores.
 constexpr int UNPACK_WG = 2;
-static_assert(A_SLOTS % UNPACK_WG == 0, "each warpgroup owns fixed TMEM slots");
-// The unpack warps reuse A slot it % A_SLOTS once the stage barrier of
-// iteration it - A_SLOTS has flipped; that barrier is not reused before
-// iteration it - A_SLOTS + STAGES >= it, which cannot have run yet.
-static_assert(STAGES >= A_SLOTS, "A-slot reuse waits on a stage barrier");
 static_assert(BK % XBOX == 0 && XBOX % MMA_K == 0, "activation boxes hold whole MMA k steps");
 constexpr int FIRST_UNPACK_WARP = 4;
 constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + 4 * UNPACK_WG;
@@ -67,11 +67,11 @@ constexpr int W_TILE_BYTES = BM * BK / 2;
 
 template <int BT>
 struct alignas(1024) Smem {
-    uint8_t act[STAGES][BT * BK];        // activation tiles: BK / XBOX boxes of [BT][128 B], 128B-swizzled
-    uint8_t wpk[STAGES][W_TILE_BYTES];   // packed weight tiles [BM][128 B], 128B-swizzled
-    uint64_t full[STAGES];               // TMA landed (tx-count barrier)
-    uint64_t empty[STAGES];              // MMAs reading the stage finished
-    uint64_t aready[A_SLOTS];            // A slot written to TMEM (4 unpack warps)
+    uint8_t act[Ring<BT>::STAGES][BT * BK];       // activation tiles: BK / XBOX boxes of [BT][128 B], 128B-swizzled
+    uint8_t wpk[Ring<BT>::STAGES][W_TILE_BYTES];  // packed weight tiles [BM][128 B], 128B-swizzled
+    uint64_t full[Ring<BT>::STAGES];              // TMA landed (tx-count barrier)
+    uint64_t empty[Ring<BT>::STAGES];             // MMAs reading the stage finished
+    uint64_t aready[Ring<BT>::A_SLOTS];           // A slot written to TMEM (4 unpack warps)
     uint64_t acc_full[2];                // accumulator ready for the epilogue
     uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
     uint64_t mma_done;                   // final drain of the MMA pipe
@@ -151,6 +151,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
           int M, int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
           const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+    constexpr int STAGES = Ring<BT>::STAGES;
+    constexpr int A_SLOTS = Ring<BT>::A_SLOTS;
+    static_assert(A_SLOTS % UNPACK_WG == 0, "each warpgroup owns fixed TMEM slots");
+    // The unpack warps reuse A slot it % A_SLOTS once the stage barrier of
+    // iteration it - A_SLOTS has flipped; that barrier is not reused before
+    // iteration it - A_SLOTS + STAGES >= it, which cannot have run yet.
+    static_assert(STAGES >= A_SLOTS, "A-slot reuse waits on a stage barrier");
     static_assert(2 * BT + A_SLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
     extern __shared__ uint8_t smem_raw[];
@@ -518,19 +525,51 @@ inline bool tc_supported(int M, int K, int N) {
 
 // act_perm: the INT8 activations use the k-permuted layout k_act_quant
 // writes for this kernel (only inside w4a8_linear's workspace).
+namespace tc {
+// Token tile for a call: the one with the smallest estimated time, where a
+// round of tiles over the SMs costs ceil(K / BK) iterations of about
+// 8 x BT / 2 tensor cycles plus ~600 cycles of per-iteration overhead.
+inline int pick_token_tile(int M, int N, int sm_count) {
+    const int cand[3] = {192, 128, 64};
+    int best = 192;
+    long long best_cost = -1;
+    for (int bt : cand) {
+        const long long tiles = (long long)((M + bt - 1) / bt) * ((N + BM - 1) / BM);
+        const long long rounds = (tiles + sm_count - 1) / sm_count;
+        const long long cost = rounds * (8LL * bt / 2 + 600);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bt;
+        }
+    }
+    return best;
+}
+
+template <int UNPACK>
+inline w4a8_status launch_bt(int bt, const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp,
+                             int ldp, const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                             int sm_count, cudaStream_t stream) {
+    if (bt == 64) return launch<64, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+    if (bt == 128)
+        return launch<128, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+    return launch<192, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+}
+}  // namespace tc
+
 inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp,
                                   int ldp, const float *sw, int N, const float *bias, unsigned flags, void *Y,
                                   int ldy, int sm_count, cudaStream_t stream, bool act_perm = false) {
+    const int bt = tc::pick_token_tile(M, N, sm_count);
     if (K > tc::TC_X16_MAX_K) {
         if (act_perm) return W4A8_ERR_UNSUPPORTED;
-        return tc::launch<tc::BT_TILE, tc::UNPACK_SEXT>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
-                                                stream);
+        return tc::launch_bt<tc::UNPACK_SEXT>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
+                                              stream);
     }
     if (act_perm)
-        return tc::launch<tc::BT_TILE, tc::UNPACK_X16_PERM>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
-                                                    sm_count, stream);
-    return tc::launch<tc::BT_TILE, tc::UNPACK_X16>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
-                                           stream);
+        return tc::launch_bt<tc::UNPACK_X16_PERM>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+                                                  sm_count, stream);
+    return tc::launch_bt<tc::UNPACK_X16>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
+                                         stream);
 }
 
 }  // namespace w4a8
