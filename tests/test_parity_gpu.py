@@ -409,3 +409,22 @@ def test_static_weights_promise_gives_same_bits(nat, m):
     q1 = host(nat.w4a8_linear_q(xq, sx, k, wpd, swd, bias=bd, static_weights=True))
     assert np.array_equal(q0.view(np.uint32), q1.view(np.uint32))
     assert np.array_equal(y0.view(np.uint32), q0.view(np.uint32))
+
+
+@pytest.mark.parametrize("m", [2, 3, 4])
+def test_fused_two_pass_decode_sampled(nat, m):
+    """Few rows against a long weight stream (K = 8192, N = 28672): the decode
+    kernel quantizes X in two passes of its own; sampled channels against the
+    oracle, plus bit-equality with quantizing first (a8_quantize_rows) and
+    multiplying after (w4a8_linear_q)."""
+    c0 = synth.llama70_case(0, 1, with_x=False)
+    k, n = synth.LLAMA70_SHAPES[0]
+    wpd, swd = nat.w4_quantize_pack(dev(c0.w))
+    x, _ = synth.linear_activations(m, k, seed=1400 + m, outlier_count=8, outlier_factor=50.0)
+    rng = synth.rng_for(14, m)
+    cols = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, size=40)]))
+    y = _sampled_check(nat, x, None, wpd, swd, np.arange(m), cols, path="decode")
+    assert nat.last_launch_count() == 1
+    xq, sx = nat.a8_quantize_rows(dev(x))
+    yq = host(nat.w4a8_linear_q(xq, sx, k, wpd, swd, path="decode"))
+    assert np.array_equal(np.asarray(y).view(np.uint32), yq.view(np.uint32))

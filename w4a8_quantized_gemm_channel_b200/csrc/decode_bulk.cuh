@@ -153,6 +153,79 @@ __device__ __forceinline__ void quantize_rows(const float *X, int ldx, int vec4,
     ptx::bar_sync(1, CONSUMERS);
 }
 
+// The same quantization for rows whose values do not fit the registers (any
+// K the stages cover): pass 1 reduces each row's abs-max while streaming X
+// (up to 4 units of 8 floats per row in flight per thread), pass 2 reads X
+// again - L1/L2-resident by then - and writes the codes.
+template <int R>
+__device__ __forceinline__ void quantize_rows_2pass(const float *X, int ldx, int vec4, int rows, int K, int ks,
+                                                    int pitch, int8_t *xs, Smem &sm, int tid, int lane, int warp) {
+    float am[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) am[r] = 0.0f;
+    auto load8 = [&](int r, int k, float (&v)[8]) {
+#pragma unroll
+        for (int b = 0; b < 8; ++b) v[b] = 0.0f;
+        if (r >= rows || k >= K) return;
+        const float *x = X + (size_t)r * ldx + k;
+        if (vec4 && k + 7 < K) {
+            const float4 f0 = ld_dep_f4(x), f1 = ld_dep_f4(x + 4);
+            v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+            v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+        } else {
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                if (k + b < K) v[b] = ld_dep(x + b);
+        }
+    };
+    constexpr int UNR = R >= 4 ? 1 : 4 / R;  // units per row in flight
+    for (int k0 = 8 * tid; k0 < K; k0 += 8 * CONSUMERS * UNR) {
+        float v[UNR][R][8];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u)
+#pragma unroll
+            for (int r = 0; r < R; ++r) load8(r, k0 + 8 * CONSUMERS * u, v[u][r]);
+#pragma unroll
+        for (int u = 0; u < UNR; ++u)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) am[r] = fmaxf(am[r], fabsf(v[u][r][b]));
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am[r] = fmaxf(am[r], __shfl_xor_sync(0xffffffffu, am[r], o));
+        if (lane == 0) sm.part[r][warp] = am[r];
+    }
+    ptx::bar_sync(1, CONSUMERS);
+    float sc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float a = sm.part[r][0];
+#pragma unroll
+        for (int w = 1; w < CONSUMER_WARPS; ++w) a = fmaxf(a, sm.part[r][w]);
+        sc[r] = act_scale_from_amax(a);
+        if (tid == 0 && r < rows) sm.sxs[r] = sc[r];
+    }
+    for (int k0 = 8 * tid; k0 < ks; k0 += 8 * CONSUMERS * UNR) {
+        float v[UNR][R][8];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u)
+#pragma unroll
+            for (int r = 0; r < R; ++r) load8(r, k0 + 8 * CONSUMERS * u, v[u][r]);
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int k = k0 + 8 * CONSUMERS * u;
+            if (k >= ks) continue;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                if (r < rows) *reinterpret_cast<uint2 *>(xs + r * pitch + k) = act_codes8_perm(v[u][r], sc[r], k, K);
+        }
+    }
+    ptx::bar_sync(1, CONSUMERS);
+}
+
 // Copy INT8 activation rows (natural order, row stride ldq) into xs in the
 // permuted order, 16 bytes per load; k from min(ldq, ks) on reads as 0.
 __device__ __forceinline__ void stage_rows(const int8_t *Xq, int ldq, int rows, int ks, int pitch, int8_t *xs,
@@ -178,7 +251,8 @@ __device__ __forceinline__ void stage_rows(const int8_t *Xq, int ldq, int rows, 
 // EARLY: the weights are final at launch (behind the activation pass, or
 // W4A8_STATIC_WEIGHTS), so the ring is filled before the dependency wait;
 // otherwise the first stages are only prefetched into L2 before it.
-// FUSED: the block quantizes X itself (M <= R, ks <= 2048 J8); otherwise
+// FUSED: the block quantizes X itself (M <= R): with the values held in
+// registers when ks <= 2048 J8, in two passes over X when J8 = 0; otherwise
 // Xq / sx come from the activation pass or the caller.
 template <bool EARLY, bool FUSED, int R, int J8>
 __global__ void __launch_bounds__(THREADS, 3)
@@ -260,7 +334,10 @@ k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ld
     griddep_wait();
     float e_sx = 1.0f;
     if constexpr (FUSED) {
-        quantize_rows<R, J8>(X, ldx, vec4, rows, K, ks, pitch, xs, sm, threadIdx.x, lane, warp);
+        if constexpr (J8 > 0)
+            quantize_rows<R, J8>(X, ldx, vec4, rows, K, ks, pitch, xs, sm, threadIdx.x, lane, warp);
+        else
+            quantize_rows_2pass<R>(X, ldx, vec4, rows, K, ks, pitch, xs, sm, threadIdx.x, lane, warp);
         if (e_row) e_sx = sm.sxs[e_tk];
     } else {
         if (e_row) e_sx = ld_dep(sx + e_tk);

@@ -208,9 +208,12 @@ cudaError_t launch_ring_q(const RingPlan &plan, bool early, const int8_t *Xq, in
                                                         flags, Y, ldy, s);
 }
 
-// Decode with the activation quantization fused in: the block keeps R rows
-// x J8 units of 8 floats per thread in registers (R * J8 <= 4), so M <= R and
-// the stages' k <= 2048 J8.
+// Decode with the activation quantization fused in, for M <= 4: the block
+// keeps R rows x J8 units of 8 floats per thread in registers when
+// R * J8 <= 4 (M <= R, the stages' k <= 2048 J8), else it reads X twice.
+// Every block reads all of X, so the two-pass form is taken only where that
+// traffic (grid x M x K x 8 bytes) stays within the weight stream (N x K / 2
+// bytes); otherwise the activation pass runs first.
 int fq_rows(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 int fq_j8(int K) {  // units per row and thread to cover the stages' k, rounded up to a power of 2
     const int j = (dbulk::Geometry(K).pitch - 16 + 2047) / 2048;
@@ -218,8 +221,11 @@ int fq_j8(int K) {  // units per row and thread to cover the stages' k, rounded 
     while (p < j) p *= 2;
     return p;
 }
+bool fq_in_registers(int M, int K) { return fq_rows(M) * fq_j8(K) <= 4; }
 bool fq_eligible(int M, int K, int N, unsigned path) {
-    return path == W4A8_PATH_DECODE && ring_plan(M, K, N).ok && fq_rows(M) * fq_j8(K) <= 4;
+    if (path != W4A8_PATH_DECODE || M > 4) return false;
+    const RingPlan plan = ring_plan(M, K, N);
+    return plan.ok && (fq_in_registers(M, K) || (long long)plan.grid * M * 16 <= N);
 }
 
 w4a8_status launch_fq(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp,
@@ -233,10 +239,20 @@ w4a8_status launch_fq(const float *X, int M, int K, int ldx, const uint8_t *Wp, 
     if (early == E && fq_rows(M) == R && fq_j8(K) == J)                                                        \
         e = launch_ring_kernel<E, true, R, J>(plan, nullptr, 0, nullptr, X, ldx, vec4, M, K, Wp, ldp, sw, N, \
                                                     bias, flags, Y, ldy, s);
-    W4A8_FQ(true, 1, 1) W4A8_FQ(true, 1, 2) W4A8_FQ(true, 1, 4) W4A8_FQ(true, 2, 1) W4A8_FQ(true, 2, 2)
-    W4A8_FQ(true, 4, 1)
-    W4A8_FQ(false, 1, 1) W4A8_FQ(false, 1, 2) W4A8_FQ(false, 1, 4) W4A8_FQ(false, 2, 1) W4A8_FQ(false, 2, 2)
-    W4A8_FQ(false, 4, 1)
+    if (fq_in_registers(M, K)) {
+        W4A8_FQ(true, 1, 1) W4A8_FQ(true, 1, 2) W4A8_FQ(true, 1, 4) W4A8_FQ(true, 2, 1) W4A8_FQ(true, 2, 2)
+        W4A8_FQ(true, 4, 1)
+        W4A8_FQ(false, 1, 1) W4A8_FQ(false, 1, 2) W4A8_FQ(false, 1, 4) W4A8_FQ(false, 2, 1) W4A8_FQ(false, 2, 2)
+        W4A8_FQ(false, 4, 1)
+    } else {  // J8 = 0: two passes over X
+#define W4A8_FQ2(E, R)                                                                                          \
+    if (early == E && fq_rows(M) == R)                                                                          \
+        e = launch_ring_kernel<E, true, R, 0>(plan, nullptr, 0, nullptr, X, ldx, vec4, M, K, Wp, ldp, sw, N, bias, \
+                                              flags, Y, ldy, s);
+        W4A8_FQ2(true, 1) W4A8_FQ2(true, 2) W4A8_FQ2(true, 4)
+        W4A8_FQ2(false, 1) W4A8_FQ2(false, 2) W4A8_FQ2(false, 4)
+#undef W4A8_FQ2
+    }
 #undef W4A8_FQ
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
     t_last_path = W4A8_PATH_DECODE;
