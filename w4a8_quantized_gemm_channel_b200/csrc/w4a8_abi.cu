@@ -384,16 +384,26 @@ static w4a8_status launch_act_quant(const float *X, int M, int K, int ldx, int8_
     const int vec4 = aligned16(X) && (ldx % 4 == 0);
     const int grid = M < 65535 ? M : 65535;
     cudaError_t e;
+    // One block per row. With few rows (fewer than two per SM) a long row
+    // gets a 1024-thread block that holds it in registers up to K = 32768;
+    // many rows keep 256-thread blocks, several per SM, and read a long row
+    // twice.
+    const bool wide = K > 4096 && M < 2 * device_info().sm_count;
     if (perm) {
         if (K <= 1024)
             e = launch_pdl(k_act_quant<128, 8, true>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
-        else
+        else if (!wide)
             e = launch_pdl(k_act_quant<256, 16, true>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+        else
+            e = launch_pdl(k_act_quant<1024, 32, true>, dim3(grid), dim3(1024), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
     } else {
         if (K <= 1024)
             e = launch_pdl(k_act_quant<128, 8, false>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
-        else
+        else if (!wide)
             e = launch_pdl(k_act_quant<256, 16, false>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+        else
+            e = launch_pdl(k_act_quant<1024, 32, false>, dim3(grid), dim3(1024), 0, s, X, M, K, ldx, Xq, ldq, sx,
+                           vec4);
     }
     return from_cuda(e);
 }
