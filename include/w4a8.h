@@ -193,6 +193,19 @@ W4A8_API unsigned w4a8_last_path(void);
  * if that call had M == 0). */
 W4A8_API unsigned w4a8_last_launch_count(void);
 
+/*
+ * w4a8_selftest_timeout - exercises the library's failure path without
+ * faulting the GPU. Every wait inside the kernels is bounded: after about a
+ * second of SM cycles it gives up, records W4A8_ERR_TIMEOUT in the device
+ * status word (the first recorded fault is kept) and the kernel returns, so
+ * the context stays usable. This call enqueues one tiny kernel whose single
+ * wait can never be satisfied, with a limit of `cycles` SM cycles
+ * (1000 <= cycles <= 2e9, else W4A8_ERR_INVALID_ARG); read the outcome with
+ * w4a8_get_device_status. For tests of the error path; the pages have no
+ * counterpart.
+ */
+W4A8_API w4a8_status w4a8_selftest_timeout(long long cycles, void *stream);
+
 /* Read (and with clear != 0, reset) the current device's status word, which
  * kernels set on an internal fault. Synchronizes `stream` first. */
 W4A8_API w4a8_status w4a8_get_device_status(int clear, void *stream);

@@ -98,3 +98,19 @@ def test_no_device_means_unsupported_not_a_crash():
         pytest.skip("a device is present")
     from w4a8_quantized_gemm_channel_b200 import native
     assert _linear(native.lib) == 2
+
+
+def test_last_launch_count_starts_at_zero_per_thread():
+    import threading
+    from w4a8_quantized_gemm_channel_b200 import native
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(native.last_launch_count()))
+    t.start()
+    t.join()
+    assert seen == [0]
+
+
+def test_selftest_timeout_rejects_bad_limits():
+    from w4a8_quantized_gemm_channel_b200 import native
+    assert native.lib.w4a8_selftest_timeout(10, None) == native.ERR_INVALID_ARG
+    assert native.lib.w4a8_selftest_timeout(10 ** 12, None) == native.ERR_INVALID_ARG

@@ -428,3 +428,18 @@ def test_fused_two_pass_decode_sampled(nat, m):
     xq, sx = nat.a8_quantize_rows(dev(x))
     yq = host(nat.w4a8_linear_q(xq, sx, k, wpd, swd, path="decode"))
     assert np.array_equal(np.asarray(y).view(np.uint32), yq.view(np.uint32))
+
+
+def test_bounded_wait_gives_up_and_reports(nat):
+    """Failure detection without a GPU fault: a wait that nothing satisfies
+    gives up after its limit, the device status word reads W4A8_ERR_TIMEOUT,
+    and the context keeps working."""
+    nat.get_device_status(clear=True)
+    nat.selftest_timeout(1_000_000)
+    assert nat.get_device_status(clear=True) == nat.ERR_TIMEOUT
+    assert nat.get_device_status() == nat.OK
+    m, k, n = 3, 64, 16
+    x, w, _ = _case(m, k, n, seed=1500)
+    wp, sw = oracle.w4_quantize_pack(w)
+    acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32")
+    assert np.array_equal(host(acc), oracle.linear(x, wp, sw, k, out="s32"))

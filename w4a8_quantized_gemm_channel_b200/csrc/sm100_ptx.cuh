@@ -60,13 +60,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // an error status instead of hanging the GPU.
 constexpr long long WAIT_LIMIT_CYCLES = 2000000000LL;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          long long limit = WAIT_LIMIT_CYCLES) {
     if (mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > limit) {
             *abort = 1;
             record_fault(W4A8_ERR_TIMEOUT);
             return false;

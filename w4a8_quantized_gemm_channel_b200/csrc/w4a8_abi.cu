@@ -304,6 +304,21 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     return W4A8_OK;
 }
 
+// Self-test of the failure path: one thread waits on an mbarrier that no one
+// arrives on; the bounded wait gives up after `limit` cycles, records
+// W4A8_ERR_TIMEOUT in the device status word and the kernel returns.
+__global__ void k_selftest_timeout(long long limit) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)ptx::mbar_wait(&bar, 0, &abort_flag, limit);
+}
+
 // Scratch of w4a8_linear_noalloc: a file-scope device array, so callers that
 // cannot allocate still get somewhere to keep the INT8 activations.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_BYTES];
@@ -482,6 +497,13 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
 unsigned w4a8_last_path(void) { return t_last_path; }
 
 unsigned w4a8_last_launch_count(void) { return t_last_launches; }
+
+w4a8_status w4a8_selftest_timeout(long long cycles, void *stream) {
+    if (cycles < 1000 || cycles > ptx::WAIT_LIMIT_CYCLES) return W4A8_ERR_INVALID_ARG;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    k_selftest_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(cycles);
+    return from_cuda(cudaGetLastError());
+}
 
 w4a8_status w4a8_get_device_status(int clear, void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);

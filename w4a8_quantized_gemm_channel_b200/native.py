@@ -41,6 +41,7 @@ SIGNATURES = {
     "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_last_path": (_U, []),
     "w4a8_last_launch_count": (_U, []),
+    "w4a8_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
     "w4a8_get_device_status": (_I, [_I, _P]),
     "w4a8_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -209,6 +210,11 @@ def last_path() -> str:
 
 def last_launch_count() -> int:
     return lib.w4a8_last_launch_count()
+
+
+def selftest_timeout(cycles: int = 1_000_000, stream=None):
+    """Enqueue the bounded-wait self-test (see include/w4a8.h)."""
+    _check(lib.w4a8_selftest_timeout(cycles, _stream(stream)), "w4a8_selftest_timeout")
 
 
 def get_device_status(clear: bool = False, stream=None) -> int:
