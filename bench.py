@@ -525,6 +525,135 @@ def run_sweep(torch, native, synth, device, props):
         torch.cuda.empty_cache()
 
 
+def run_gemma_stack(torch, native, synth, device, steps=20):
+    """The Gemma3-1B-shaped stack: 26 layers x 7 projections = 182 independent
+    linears (distinct quantized weights, 349 MB packed), run back to back in
+    one CUDA graph per M, with the static-weights promise. One JSON line per
+    M with the aggregate and per-projection-type rates; the roofline fraction
+    is max(T_mem, T_tc) / T_measured over the algorithmic bytes and ops."""
+    peaks, _ = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    tc = INT8_OVER_BF16 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    layers = []
+    for layer in range(synth.GEMMA_LAYERS):
+        row = []
+        for p in range(len(synth.GEMMA_PROJ)):
+            w = torch.from_numpy(synth.gemma_weights(layer, p)).to(device)
+            row.append(native.w4_quantize_pack(w))
+            del w
+        layers.append(row)
+    torch.cuda.synchronize()
+
+    def timed_graph(calls):
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for c in calls:
+                c()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            g.replay()
+        stop.record()
+        torch.cuda.synchronize()
+        return start.elapsed_time(stop) * 1e3 / steps  # us per replay
+
+    for m in synth.GEMMA_MS:
+        xs = [torch.from_numpy(synth.gemma_activations(m, k, sub=p)).to(device)
+              for p, (_, k, _) in enumerate(synth.GEMMA_PROJ)]
+        ys = [torch.empty((m, n), dtype=torch.float32, device=device) for (_, _, n) in synth.GEMMA_PROJ]
+        wss = [torch.empty(native.workspace_size(m, k), dtype=torch.uint8, device=device)
+               for (_, k, _) in synth.GEMMA_PROJ]
+
+        def call(layer, p):
+            wp, sw = layers[layer][p]
+            return lambda: native.w4a8_linear(xs[p], wp, sw, y=ys[p], workspace=wss[p], static_weights=True)
+
+        def work(ps):
+            nbytes = ops = 0
+            for p in ps:
+                _, k, n = synth.GEMMA_PROJ[p]
+                nbytes += synth.GEMMA_LAYERS * (n * native.packed_ld(k) + 4 * n + 4 * m * k + 4 * m * n)
+                ops += synth.GEMMA_LAYERS * 2 * m * n * k
+            return nbytes, ops
+
+        def rates(us, ps):
+            nbytes, ops = work(ps)
+            t_mem, t_tc = nbytes / (hbm * 1e3), ops / (tc * 1e6)  # us at the peaks
+            return {"us": round(us, 2), "GBs": round(nbytes / (us * 1e3), 1),
+                    "TOPS": round(ops / (us * 1e6), 2), "roofline_frac": round(max(t_mem, t_tc) / us, 4)}
+
+        all_p = range(len(synth.GEMMA_PROJ))
+        us_all = timed_graph([call(layer, p) for layer in range(synth.GEMMA_LAYERS) for p in all_p])
+
+        # The same 182 linears with a transformer layer's dependency structure
+        # instead of one serial chain: q, k, v on three streams, then o, then
+        # gate and up on two streams, then down (fork and join through events
+        # inside the one graph). Outputs of parallel branches go to distinct
+        # buffers, so the branches share no memory.
+        side = [torch.cuda.Stream(device=device) for _ in range(2)]
+
+        def branches(layer, group):
+            main = torch.cuda.current_stream()
+            for st in side[:len(group) - 1]:
+                st.wait_stream(main)
+            for st, p in zip([main] + side, group):
+                with torch.cuda.stream(st):
+                    call(layer, p)()
+            for st in side[:len(group) - 1]:
+                main.wait_stream(st)
+
+        def layered():
+            for layer in range(synth.GEMMA_LAYERS):
+                branches(layer, [0, 1, 2])  # q, k, v
+                call(layer, 3)()            # o
+                branches(layer, [4, 5])     # gate, up
+                call(layer, 6)()            # down
+        us_dep = timed_graph([layered])
+
+        # All 182 linears as one grouped call (M <= 4 only): persistent
+        # launches of up to 64 problems each instead of 182 launches.
+        us_grp = None
+        if m <= 4:
+            probs = [(xs[p], layers[layer][p][0], layers[layer][p][1], None)
+                     for layer in range(synth.GEMMA_LAYERS) for p in all_p]
+            outs = [torch.empty((m, synth.GEMMA_PROJ[p][2]), dtype=torch.float32, device=device)
+                    for p in all_p]
+            arr = (native.Problem * len(probs))()
+            for i, (x, wp, sw, _) in enumerate(probs):
+                n = wp.shape[0]
+                y = outs[i % len(outs)]
+                arr[i] = native.Problem(x.data_ptr(), wp.data_ptr(), sw.data_ptr(), None, y.data_ptr(),
+                                        m, x.shape[1], x.stride(0), wp.stride(0), n, y.stride(0))
+            flags = native.flags_for(static_weights=True)
+
+            def grouped():
+                rc = native.lib.w4a8_linear_grouped(arr, len(probs), flags,
+                                                   native._stream(torch.cuda.current_stream()))
+                assert rc == native.OK, rc
+            us_grp = timed_graph([grouped])
+        per_type = {}
+        for p, (nm, _, _) in enumerate(synth.GEMMA_PROJ):
+            us_p = timed_graph([call(layer, p) for layer in range(synth.GEMMA_LAYERS)])
+            per_type[nm] = rates(us_p, [p])
+        print(json.dumps({"workload": "gemma3-1b-shaped stack, 26 layers x 7 linears in one CUDA graph",
+                          "M": m, "aggregate": rates(us_all, list(all_p)),
+                          "aggregate_layer_dependencies": rates(us_dep, list(all_p)),
+                          "aggregate_grouped": rates(us_grp, list(all_p)) if us_grp else None,
+                          "per_type": per_type, "call": "w4a8_linear with W4A8_STATIC_WEIGHTS",
+                          "note": "aggregate: one serial chain of 182 calls; aggregate_layer_dependencies: "
+                                  "q/k/v and gate/up as parallel branches, o and down after them; "
+                                  "aggregate_grouped: the 182 independent linears through "
+                                  "w4a8_linear_grouped (one launch per 64)"}),
+              flush=True)
+        del xs, ys, wss
+
+
 # --------------------------------------------------------------- main ---
 
 def main():
@@ -535,10 +664,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU work for the oracle baseline")
-    ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep"],
+    ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep", "gemma-stack"],
                     default="decode",
-                    help="decode (the headline line), prefill (M=2048 K=4096 N=11008), "
-                         "or a per-shape sweep of the other workloads")
+                    help="decode (the headline line), prefill (M=2048 K=4096 N=11008), a per-shape "
+                         "sweep of the other workloads, or the 182-linear Gemma3-1B-shaped stack")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -579,6 +708,9 @@ def main():
         return
     if args.workload == "sweep":
         run_sweep(torch, native, synth, device, props)
+        return
+    if args.workload == "gemma-stack":
+        run_gemma_stack(torch, native, synth, device)
         return
     wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size)
 

@@ -184,6 +184,34 @@ W4A8_API w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx,
                                          const float *bias, unsigned flags,
                                          void *Y, int ldy, void *stream);
 
+/*
+ * w4a8_linear_grouped - many independent few-row linears (steps 3-6 each) in
+ * as few launches as possible: one persistent launch per 64 problems. Meant
+ * for batches of small layers whose separate launches would each pay the
+ * dependency latency of a kernel: the projections of a model that do not
+ * feed each other, or the experts of a mixture-of-experts layer at decode.
+ * The pages have no counterpart; each problem's output holds the same bits as
+ * w4a8_linear on that problem alone.
+ *   probs[i]: X [M][ldx] float32 with 0 <= M <= 4 (M == 0: nothing to do),
+ *       Wp [N][ldp] and sw [N] as from w4_quantize_pack, bias [N] or NULL,
+ *       Y [M][ldy] in the W4A8_OUT_* format of `flags`; per-problem argument
+ *       rules as for w4a8_linear. The array is read during the call only.
+ *   flags: W4A8_RELU | one W4A8_OUT_* | W4A8_STATIC_WEIGHTS, for every problem.
+ * Returns W4A8_ERR_UNSUPPORTED when a problem's INT8 rows do not fit a
+ * block's shared memory (M x round_up(K, 4096) + 16 bytes beyond about
+ * 68 KB); nothing is enqueued then. No workspace is needed.
+ */
+typedef struct w4a8_problem {
+    const float *X;
+    const uint8_t *Wp;
+    const float *sw;
+    const float *bias;
+    void *Y;
+    int M, K, ldx, ldp, N, ldy;
+} w4a8_problem;
+
+W4A8_API w4a8_status w4a8_linear_grouped(const w4a8_problem *probs, int count, unsigned flags, void *stream);
+
 /* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
  * last successful w4a8_linear / w4a8_linear_q call enqueued; 0 if none. */
 W4A8_API unsigned w4a8_last_path(void);

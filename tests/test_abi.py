@@ -114,3 +114,16 @@ def test_selftest_timeout_rejects_bad_limits():
     from w4a8_quantized_gemm_channel_b200 import native
     assert native.lib.w4a8_selftest_timeout(10, None) == native.ERR_INVALID_ARG
     assert native.lib.w4a8_selftest_timeout(10 ** 12, None) == native.ERR_INVALID_ARG
+
+
+def test_grouped_rejects_bad_arguments_before_the_device():
+    import ctypes as ct
+    from w4a8_quantized_gemm_channel_b200 import native
+    P = native.Problem
+    assert native.lib.w4a8_linear_grouped(None, 0, 0, None) == native.OK        # nothing to do
+    assert native.lib.w4a8_linear_grouped(None, 1, 0, None) == native.ERR_INVALID_ARG
+    arr = (P * 1)(P(16, 4096, 8192, None, 12288, 5, 64, 64, 32, 8, 8))     # M = 5 > 4
+    assert native.lib.w4a8_linear_grouped(arr, 1, 0, None) == native.ERR_INVALID_ARG
+    arr = (P * 1)(P(16, 4096, 8192, None, 12288, 2, 64, 64, 32, 8, 8))
+    assert native.lib.w4a8_linear_grouped(arr, 1, native.PATH_TC, None) == native.ERR_INVALID_ARG
+    assert ct.sizeof(P) == 64

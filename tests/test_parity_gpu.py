@@ -443,3 +443,53 @@ def test_bounded_wait_gives_up_and_reports(nat):
     wp, sw = oracle.w4_quantize_pack(w)
     acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32")
     assert np.array_equal(host(acc), oracle.linear(x, wp, sw, k, out="s32"))
+
+
+# ------------------------------------------------------ grouped decode ---
+
+def _grouped_case(specs, seed):
+    probs, refs = [], []
+    for i, (m, k, n, with_bias) in enumerate(specs):
+        x, w, b = _case(m, k, n, seed=seed + i)
+        if m > 1:
+            x[m - 1] = 0.0                     # an all-zero row
+        wp, sw = oracle.w4_quantize_pack(w)
+        probs.append((x, wp, sw, b if with_bias else None))
+    return probs
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16", "s32"])
+def test_grouped_decode_matches_single_calls(nat, out):
+    """Heterogeneous problems (K from 1 to 6912, odd K, N tails, M 1..4, some
+    with a bias) in one grouped call give the same bits as one w4a8_linear per
+    problem, and the INT32 accumulators equal the oracle's."""
+    specs = [(1, 4096, 4096, True), (4, 1152, 1024, False), (2, 7, 40, True), (3, 6912, 1152, True),
+             (1, 1, 17, False), (4, 4100, 300, True), (1, 1152, 256, False), (2, 999, 96, False)]
+    probs = _grouped_case(specs, seed=1600)
+    relu = out != "s32"
+    dp = [(dev(x), dev(wp), dev(sw), None if (b is None or out == "s32") else dev(b)) for x, wp, sw, b in probs]
+    ys = nat.w4a8_linear_grouped(dp, relu=relu, out=out)
+    assert nat.last_launch_count() == 1
+    for (x, wp, sw, b), (xd, wpd, swd, bd), y in zip(probs, dp, ys):
+        y1 = nat.w4a8_linear(xd, wpd, swd, bias=bd, relu=relu, out=out)
+        a = host(y.view(torch.int32) if out != "bf16" else y.view(torch.int16))
+        b1 = host(y1.view(torch.int32) if out != "bf16" else y1.view(torch.int16))
+        assert np.array_equal(a, b1)
+        if out == "s32":
+            assert np.array_equal(host(y), oracle.linear(x, wp, sw, x.shape[1], out="s32"))
+
+
+def test_grouped_decode_many_problems_and_static_weights(nat):
+    """More problems than one launch holds (70 of them), M = 0 problems
+    skipped, and the static-weights promise: same bits as single calls."""
+    specs = [((i % 4) + 1, 64 * (1 + i % 9), 16 * (1 + i % 5) + (i % 3), i % 2 == 0) for i in range(70)]
+    probs = _grouped_case(specs, seed=1700)
+    dp = [(dev(x), dev(wp), dev(sw), None if b is None else dev(b)) for x, wp, sw, b in probs]
+    empty = (torch.empty((0, 64), device="cuda"), dp[0][1], dp[0][2], None)
+    torch.cuda.synchronize()
+    ys = nat.w4a8_linear_grouped(dp[:35] + [empty] + dp[35:], static_weights=True)
+    assert nat.last_launch_count() == 2
+    ys = ys[:35] + ys[36:]
+    for (xd, wpd, swd, bd), y in zip(dp, ys):
+        y1 = nat.w4a8_linear(xd, wpd, swd, bias=bd)
+        assert np.array_equal(host(y).view(np.uint32), host(y1).view(np.uint32))

@@ -245,6 +245,60 @@ __device__ __forceinline__ void stage_rows(const int8_t *Xq, int ldq, int rows, 
     ptx::bar_sync(1, CONSUMERS);
 }
 
+// MMAs of one stage: this warp's 64-byte chunks c = warp, warp + 8, ... of
+// the 16 rows x sb bytes at `st` (already offset by 16 t) against the INT8
+// rows (xrow = this thread's row g at byte 32 t; stage s covers
+// k in [2 sb s, 2 sb (s + 1))). Four accumulators (one per word of a piece)
+// keep the MMAs in four short dependency chains.
+__device__ __forceinline__ void stage_mma(int32_t (&acc)[4][4], const uint8_t *st, int sb, int s,
+                                          const int8_t *xrow, bool x_ok, int g, int warp) {
+    const int cps = sb / 64;
+#pragma unroll 2
+    for (int c = warp; c < cps; c += CONSUMER_WARPS) {
+        const uint4 wa = ptx::lds128(st + g * sb + 64 * c);
+        const uint4 wb = ptx::lds128(st + (g + 8) * sb + 64 * c);
+        const int8_t *xp = xrow + 2 * sb * s + 128 * c;
+        const uint4 x0 = x_ok ? ptx::lds128(xp) : make_uint4(0, 0, 0, 0);
+        const uint4 x1 = x_ok ? ptx::lds128(xp + 16) : make_uint4(0, 0, 0, 0);
+        const uint32_t pa[4] = {wa.x, wa.y, wa.z, wa.w}, pb[4] = {wb.x, wb.y, wb.z, wb.w};
+        const uint32_t xe[4] = {x0.x, x0.z, x1.x, x1.z}, xo[4] = {x0.y, x0.w, x1.y, x1.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t alo = (pa[q] << 4) & 0xF0F0F0F0u;  // 16 q of even k
+            const uint32_t ahi = pa[q] & 0xF0F0F0F0u;         // 16 q of odd k
+            const uint32_t blo = (pb[q] << 4) & 0xF0F0F0F0u;
+            const uint32_t bhi = pb[q] & 0xF0F0F0F0u;
+            mma_s8_16832(acc[q], alo, blo, ahi, bhi, xe[q], xo[q]);
+        }
+    }
+}
+
+// End of a 16-channel group: the warps' C fragments (rows g, g+8 = channels,
+// columns 2t, 2t+1 = tokens) meet in shared memory; thread e (< 16 x TOK)
+// gets the block total of output (channel e % 16, token e / 16), as 16 x the
+// product (returned shifted back). Returns false, after raising the abort
+// flag, if any consumer warp gave up; every consumer thread then agrees.
+__device__ __forceinline__ bool group_reduce(Smem &sm, int32_t (&acc)[4][4], bool ok, int warp, int g, int t,
+                                             volatile int *abort, int32_t &sum) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[0][q] += acc[1][q] + acc[2][q] + acc[3][q];
+    sm.red[warp][g][2 * t] = acc[0][0];
+    sm.red[warp][g][2 * t + 1] = acc[0][1];
+    sm.red[warp][g + 8][2 * t] = acc[0][2];
+    sm.red[warp][g + 8][2 * t + 1] = acc[0][3];
+    if (!ptx::bar_and(1, CONSUMERS, ok)) {
+        if (threadIdx.x == 0) *abort = 1;  // lets the producer stop refilling
+        return false;
+    }
+    sum = 0;
+    if (threadIdx.x < 16 * TOK) {
+#pragma unroll
+        for (int w = 0; w < CONSUMER_WARPS; ++w) sum += sm.red[w][threadIdx.x % 16][threadIdx.x / 16];
+        sum >>= 4;  // exact: every term is a multiple of 16
+    }
+    return true;
+}
+
 // tm_w: the packed weights as a [N][kp / 8] tensor of 8-byte elements with
 // row stride ldp, boxes of sb / 8 x 16. ring_n: ring slots (the host sizes
 // the dynamic shared memory as ring_n stages + the activation rows).
@@ -344,7 +398,6 @@ k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ld
         stage_rows(Xq, ldq, rows, ks, pitch, xs, threadIdx.x);
     }
 
-    const int cps = sb / 64;  // 64-byte chunks per stage
     const bool x_ok = g < rows;
     const int8_t *xrow = xs + g * pitch + 32 * t;
     bool ok = true;
@@ -356,8 +409,6 @@ k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ld
             e_sw = ld_dep(sw + n0 + e_ch);
             if (has_bias) e_b = ld_dep(bias + n0 + e_ch);
         }
-        // Four accumulators (one per word of a piece), so the MMAs form four
-        // short dependency chains instead of one long one.
         int32_t acc[4][4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0;
@@ -367,48 +418,180 @@ k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ld
                 ok = false;  // warp-uniform, so the warp leaves the loop together
                 break;
             }
-            const uint8_t *st = ring + (size_t)slot * stage_bytes + 16 * t;
-#pragma unroll 2
-            for (int c = warp; c < cps; c += CONSUMER_WARPS) {
-                const uint4 wa = ptx::lds128(st + g * sb + 64 * c);
-                const uint4 wb = ptx::lds128(st + (g + 8) * sb + 64 * c);
-                const int8_t *xp = xrow + 2 * sb * s + 128 * c;
-                const uint4 x0 = x_ok ? ptx::lds128(xp) : make_uint4(0, 0, 0, 0);
-                const uint4 x1 = x_ok ? ptx::lds128(xp + 16) : make_uint4(0, 0, 0, 0);
-                const uint32_t pa[4] = {wa.x, wa.y, wa.z, wa.w}, pb[4] = {wb.x, wb.y, wb.z, wb.w};
-                const uint32_t xe[4] = {x0.x, x0.z, x1.x, x1.z}, xo[4] = {x0.y, x0.w, x1.y, x1.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t alo = (pa[q] << 4) & 0xF0F0F0F0u;  // 16 q of even k
-                    const uint32_t ahi = pa[q] & 0xF0F0F0F0u;         // 16 q of odd k
-                    const uint32_t blo = (pb[q] << 4) & 0xF0F0F0F0u;
-                    const uint32_t bhi = pb[q] & 0xF0F0F0F0u;
-                    mma_s8_16832(acc[q], alo, blo, ahi, bhi, xe[q], xo[q]);
-                }
-            }
+            stage_mma(acc, ring + (size_t)slot * stage_bytes + 16 * t, sb, s, xrow, x_ok, g, warp);
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&sm.empty[slot]);
         }
-
-        // C fragment: rows g, g+8 (channels), columns 2t, 2t+1 (tokens)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[0][q] += acc[1][q] + acc[2][q] + acc[3][q];
-        sm.red[warp][g][2 * t] = acc[0][0];
-        sm.red[warp][g][2 * t + 1] = acc[0][1];
-        sm.red[warp][g + 8][2 * t] = acc[0][2];
-        sm.red[warp][g + 8][2 * t + 1] = acc[0][3];
-        if (!ptx::bar_and(1, CONSUMERS, ok)) {
-            if (threadIdx.x == 0) *abort = 1;  // lets the producer stop refilling
-            return;
-        }
-        if (e_ok) {
-            int32_t sum = 0;
-#pragma unroll
-            for (int w = 0; w < CONSUMER_WARPS; ++w) sum += sm.red[w][e_ch][e_tk];
-            sum >>= 4;  // exact: every term is a multiple of 16
-            store_value(Y, ldy, e_tk, n0 + e_ch, sum, e_sx, e_sw, has_bias, e_b, flags);
-        }
+        int32_t sum;
+        if (!group_reduce(sm, acc, ok, warp, g, t, abort, sum)) return;
+        if (e_ok) store_value(Y, ldy, e_tk, n0 + e_ch, sum, e_sx, e_sw, has_bias, e_b, flags);
         ptx::bar_sync(1, CONSUMERS);  // red is rewritten by the next group
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Grouped decode: many independent few-row linears in one persistent launch.
+// The problems' 16-channel groups are numbered one after another; block b
+// takes the contiguous run [T b / grid, T (b + 1) / grid) of the T groups, so
+// it switches problems rarely. Its producer streams every (group, stage) of
+// that run through one ring (slots of the largest stage, 16 x 2048 bytes)
+// with each problem's own tensor map; its consumers quantize a problem's
+// activation rows into shared memory (two passes over X, the arithmetic of
+// k_act_quant) whenever the run enters that problem, then multiply as in
+// k_decode_ring. Each problem's result is the same bits a single call gives.
+// The table travels by value in the launch parameters (tensor maps
+// included), so a captured graph holds everything it needs.
+// ---------------------------------------------------------------------------
+constexpr int MAX_GROUPED = 64;
+constexpr int GROUPED_SLOT = ROWS * MAX_STAGE_BYTES;
+
+struct GroupedProblem {
+    CUtensorMap tm;  // packed weights as [N][kp / 8] elements of 8 bytes (boxes of sb / 8 x 16)
+    const float *X;
+    const float *sw;
+    const float *bias;
+    void *Y;
+    int M, K, ldx, ldy, N, vec4, group0, pad;
+};
+struct GroupedTable {
+    GroupedProblem p[MAX_GROUPED];
+    int count;
+    int total_groups;
+};
+static_assert(sizeof(GroupedTable) <= 30 * 1024, "kernel parameter space");
+
+// Position in a block's run of (group, stage) items.
+struct GroupedCursor {
+    int gi, p, s, nst, sb;
+    __device__ __forceinline__ void enter(const GroupedTable &tab) {
+        while (p + 1 < tab.count && gi >= tab.p[p + 1].group0) ++p;
+        const Geometry geo(tab.p[p].K);
+        nst = geo.nst;
+        sb = geo.sb;
+    }
+    __device__ __forceinline__ void next(const GroupedTable &tab) {
+        if (++s == nst) {
+            s = 0;
+            ++gi;
+            enter(tab);
+        }
+    }
+};
+
+template <bool EARLY, int R>
+__global__ void __launch_bounds__(THREADS, 2)
+k_decode_grouped(const __grid_constant__ GroupedTable tab, unsigned flags, int ring_n) {
+    __shared__ Smem sm;
+    extern __shared__ __align__(1024) uint8_t dyn_smem[];
+    uint8_t *ring = dyn_smem;  // [ring_n][GROUPED_SLOT]
+    int8_t *xs = reinterpret_cast<int8_t *>(dyn_smem + (size_t)ring_n * GROUPED_SLOT);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int T = tab.total_groups;
+    const int g_begin = (int)((long long)T * blockIdx.x / gridDim.x);
+    const int g_end = (int)((long long)T * (blockIdx.x + 1) / gridDim.x);
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ring_n; ++s) {
+            ptx::mbar_init(&sm.full[s], 1);
+            ptx::mbar_init(&sm.empty[s], CONSUMER_WARPS);
+        }
+        sm.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    griddep_launch_dependents();
+    if (g_begin >= g_end) {
+        griddep_wait();
+        return;
+    }
+
+    if (warp == CONSUMER_WARPS) {
+        // ------------------------------------------------- producer (lane 0)
+        GroupedCursor cur{g_begin, 0, 0, 0, 0};
+        if (lane == 0) cur.enter(tab);
+        int issued = 0;
+        auto issue = [&]() {
+            const GroupedProblem &pr = tab.p[cur.p];
+            const int slot = issued % ring_n;
+            ptx::mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)(ROWS * cur.sb));
+            ptx::tma_load_2d(ring + (size_t)slot * GROUPED_SLOT, &pr.tm, cur.s * (cur.sb / 8),
+                             (cur.gi - pr.group0) * ROWS, &sm.full[slot]);
+            ++issued;
+            cur.next(tab);
+        };
+        if constexpr (EARLY) {
+            if (lane == 0)
+                while (issued < ring_n && cur.gi < g_end) issue();
+        }
+        // the whole warp waits together (a lane in griddepcontrol.wait holds it)
+        __syncwarp();
+        griddep_wait();
+        if (lane != 0) return;
+        bool ok = true;
+        while (ok && cur.gi < g_end) {
+            if (issued >= ring_n) {
+                const int j = issued - ring_n;  // last use of this slot
+                ok = ptx::mbar_wait(&sm.empty[j % ring_n], (uint32_t)(j / ring_n) & 1u, abort);
+                if (!ok) break;
+            }
+            issue();
+        }
+        // the block may exit only when every copy it issued has landed
+        for (int it = max(0, issued - ring_n); it < issued; ++it)
+            ptx::mbar_wait_drain(&sm.full[it % ring_n], (uint32_t)(it / ring_n) & 1u);
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    const int g = lane >> 2, t = lane & 3;
+    const int e_ch = threadIdx.x % 16, e_tk = threadIdx.x / 16;
+    const bool out_s32 = (flags & W4A8_OUT_MASK) == W4A8_OUT_S32;
+    griddep_wait();
+    GroupedCursor cur{g_begin, 0, 0, 0, 0};
+    cur.enter(tab);
+    int staged = -1, item = 0;
+    bool ok = true;
+    float e_sx = 1.0f;
+    while (cur.gi < g_end) {
+        const GroupedProblem &pr = tab.p[cur.p];
+        const Geometry geo(pr.K);
+        const int rows = pr.M;
+        if (cur.p != staged) {  // the run enters a new problem: its INT8 rows
+            quantize_rows_2pass<R>(pr.X, pr.ldx, pr.vec4, rows, pr.K, geo.pitch - 16, geo.pitch, xs, sm,
+                                   threadIdx.x, lane, warp);
+            staged = cur.p;
+            e_sx = (threadIdx.x < 16 * TOK && e_tk < rows) ? sm.sxs[e_tk] : 1.0f;
+        }
+        const int n0 = (cur.gi - pr.group0) * ROWS;
+        const bool e_ok = threadIdx.x < 16 * TOK && e_tk < rows && n0 + e_ch < pr.N;
+        const bool has_bias = pr.bias != nullptr && !out_s32;
+        float e_sw = 1.0f, e_b = 0.0f;
+        if (e_ok) {
+            e_sw = ld_dep(pr.sw + n0 + e_ch);
+            if (has_bias) e_b = ld_dep(pr.bias + n0 + e_ch);
+        }
+        int32_t acc[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0;
+        const int8_t *xrow = xs + g * geo.pitch + 32 * t;
+        const int gi = cur.gi;
+        while (ok && cur.gi == gi) {
+            const int slot = item % ring_n;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sm.full[slot], (uint32_t)(item / ring_n) & 1u, abort))) {
+                ok = false;  // warp-uniform, so the warp leaves the loop together
+                break;
+            }
+            stage_mma(acc, ring + (size_t)slot * GROUPED_SLOT + 16 * t, cur.sb, cur.s, xrow, g < rows, g, warp);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&sm.empty[slot]);
+            ++item;
+            cur.next(tab);
+        }
+        int32_t sum;
+        if (!group_reduce(sm, acc, ok, warp, g, t, abort, sum)) return;
+        if (e_ok) store_value(pr.Y, pr.ldy, e_tk, n0 + e_ch, sum, e_sx, e_sw, has_bias, e_b, flags);
+        ptx::bar_sync(1, CONSUMERS);  // red (and xs, on a problem change) are rewritten next
     }
 }
 

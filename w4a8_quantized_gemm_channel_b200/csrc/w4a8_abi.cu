@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <cstdio>
+#include <cstring>
 #include <map>
 #include <mutex>
 
@@ -304,6 +305,68 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     return W4A8_OK;
 }
 
+// One launch of the grouped decode kernel over probs[0..count) (count <= 64,
+// every M >= 1).
+template <bool EARLY, int R>
+cudaError_t launch_grouped_kernel(const dbulk::GroupedTable &tab, int grid, int ring_n, size_t smem, unsigned flags,
+                                  cudaStream_t s) {
+    auto kern = dbulk::k_decode_grouped<EARLY, R>;
+    if (!raise_smem_limit(reinterpret_cast<const void *>(kern), dbulk::SMEM_BUDGET)) return cudaErrorInvalidValue;
+    return launch_pdl(kern, dim3(grid), dim3(dbulk::THREADS), smem, s, tab, flags, ring_n);
+}
+
+w4a8_status launch_grouped_chunk(const w4a8_problem *probs, int count, unsigned flags, cudaStream_t s) {
+    static dbulk::GroupedTable tab;  // built under the lock, copied into the launch parameters
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    memset(&tab, 0, sizeof(tab));
+    int total = 0, max_m = 0, max_pitch = 0;
+    for (int i = 0; i < count; ++i) {
+        const w4a8_problem &p = probs[i];
+        const dbulk::Geometry geo(p.K);
+        dbulk::GroupedProblem &q = tab.p[i];
+        if (!tc::make_map_2d(&q.tm, CU_TENSOR_MAP_DATA_TYPE_UINT64, p.Wp, (uint64_t)(geo.kp / 8), (uint64_t)p.N,
+                             (uint64_t)p.ldp, (uint32_t)(geo.sb / 8), dbulk::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return W4A8_ERR_CUDA;
+        q.X = p.X;
+        q.sw = p.sw;
+        q.bias = p.bias;
+        q.Y = p.Y;
+        q.M = p.M;
+        q.K = p.K;
+        q.ldx = p.ldx;
+        q.ldy = p.ldy;
+        q.N = p.N;
+        q.vec4 = aligned16(p.X) && (p.ldx % 4 == 0);
+        q.group0 = total;
+        total += (p.N + dbulk::ROWS - 1) / dbulk::ROWS;
+        max_m = max_m > p.M ? max_m : p.M;
+        max_pitch = max_pitch > geo.pitch ? max_pitch : geo.pitch;
+    }
+    tab.count = count;
+    tab.total_groups = total;
+    const int r = fq_rows(max_m);
+    const long long xs = (long long)r * max_pitch;
+    const long long ring = ((long long)dbulk::SMEM_BUDGET - xs) / dbulk::GROUPED_SLOT;
+    if (ring < 1) return W4A8_ERR_UNSUPPORTED;
+    const int ring_n = (int)(ring < dbulk::MAX_RING ? ring : dbulk::MAX_RING);
+    const int sms = device_info().sm_count;
+    const int grid = total < 2 * sms ? total : 2 * sms;
+    const size_t smem = (size_t)ring_n * dbulk::GROUPED_SLOT + (size_t)xs;
+    const bool early = (flags & W4A8_STATIC_WEIGHTS) != 0;
+    cudaError_t e;
+    if (r == 1)
+        e = early ? launch_grouped_kernel<true, 1>(tab, grid, ring_n, smem, flags, s)
+                  : launch_grouped_kernel<false, 1>(tab, grid, ring_n, smem, flags, s);
+    else if (r == 2)
+        e = early ? launch_grouped_kernel<true, 2>(tab, grid, ring_n, smem, flags, s)
+                  : launch_grouped_kernel<false, 2>(tab, grid, ring_n, smem, flags, s);
+    else
+        e = early ? launch_grouped_kernel<true, 4>(tab, grid, ring_n, smem, flags, s)
+                  : launch_grouped_kernel<false, 4>(tab, grid, ring_n, smem, flags, s);
+    return from_cuda(e);
+}
+
 // Self-test of the failure path: one thread waits on an mbarrier that no one
 // arrives on; the bounded wait gives up after `limit` cycles, records
 // W4A8_ERR_TIMEOUT in the device status word and the kernel returns.
@@ -497,6 +560,46 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
 unsigned w4a8_last_path(void) { return t_last_path; }
 
 unsigned w4a8_last_launch_count(void) { return t_last_launches; }
+
+w4a8_status w4a8_linear_grouped(const w4a8_problem *probs, int count, unsigned flags, void *stream) {
+    if (count < 0 || (count > 0 && !probs)) return W4A8_ERR_INVALID_ARG;
+    if (flags & W4A8_PATH_MASK) return W4A8_ERR_INVALID_ARG;
+    bool any = false;
+    // every problem is checked before anything is enqueued
+    for (int i = 0; i < count; ++i) {
+        const w4a8_problem &p = probs[i];
+        w4a8_status st = check_common(p.M, p.K, p.N, p.Wp, p.ldp, p.sw, p.bias, flags, p.Y, p.ldy);
+        if (st != W4A8_OK) return st;
+        if (p.M > 4 || p.ldx < p.K) return W4A8_ERR_INVALID_ARG;
+        if (p.M == 0) continue;
+        any = true;
+        if (!p.X || !aligned4(p.X)) return W4A8_ERR_INVALID_ARG;
+        if (p.K > dbulk::X16_MAX_K) return W4A8_ERR_UNSUPPORTED;
+        if ((long long)fq_rows(p.M) * dbulk::Geometry(p.K).pitch + dbulk::GROUPED_SLOT > dbulk::SMEM_BUDGET)
+            return W4A8_ERR_UNSUPPORTED;
+    }
+    if (!any) {  // nothing to do
+        t_last_launches = 0;
+        return W4A8_OK;
+    }
+    if (!device_info().ok || tc::encode_fn() == nullptr) return W4A8_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned launches = 0;
+    w4a8_problem chunk[dbulk::MAX_GROUPED];
+    int n = 0;
+    for (int i = 0; i <= count; ++i) {
+        if (i < count && probs[i].M > 0) chunk[n++] = probs[i];
+        if (n == dbulk::MAX_GROUPED || (i == count && n > 0)) {
+            w4a8_status st = launch_grouped_chunk(chunk, n, flags, s);
+            if (st != W4A8_OK) return st;
+            ++launches;
+            n = 0;
+        }
+    }
+    t_last_path = W4A8_PATH_DECODE;
+    t_last_launches = launches;
+    return W4A8_OK;
+}
 
 w4a8_status w4a8_selftest_timeout(long long cycles, void *stream) {
     if (cycles < 1000 || cycles > ptx::WAIT_LIMIT_CYCLES) return W4A8_ERR_INVALID_ARG;

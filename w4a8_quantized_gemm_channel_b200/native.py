@@ -28,6 +28,14 @@ _OUT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "s32": torch.int32}
 _PATH = {"auto": PATH_AUTO, "generic": PATH_GENERIC, "decode": PATH_DECODE, "tc": PATH_TC}
 PATH_NAMES = {v: k for k, v in _PATH.items()}
 
+class Problem(ctypes.Structure):
+    """struct w4a8_problem of include/w4a8.h."""
+    _fields_ = [("X", ctypes.c_void_p), ("Wp", ctypes.c_void_p), ("sw", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("Y", ctypes.c_void_p), ("M", ctypes.c_int),
+                ("K", ctypes.c_int), ("ldx", ctypes.c_int), ("ldp", ctypes.c_int), ("N", ctypes.c_int),
+                ("ldy", ctypes.c_int)]
+
+
 # Every symbol include/w4a8.h declares, with its ctypes signature.
 _P, _I, _U, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t
 SIGNATURES = {
@@ -42,6 +50,7 @@ SIGNATURES = {
     "w4a8_last_path": (_U, []),
     "w4a8_last_launch_count": (_U, []),
     "w4a8_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
+    "w4a8_linear_grouped": (_I, [ctypes.POINTER(Problem), _I, _U, _P]),
     "w4a8_get_device_status": (_I, [_I, _P]),
     "w4a8_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -181,6 +190,27 @@ def w4a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor,
                              _stream(stream)),
            "w4a8_linear_q")
     return y
+
+
+def w4a8_linear_grouped(problems, relu: bool = False, out: str = "f32", stream=None,
+                        static_weights: bool = False):
+    """Many independent few-row linears in as few launches as possible.
+    problems: list of (x, wp, sw, bias_or_None) with x [M][K] float32, M <= 4.
+    Returns the list of outputs Y [M][N]."""
+    arr = (Problem * max(1, len(problems)))()
+    ys = []
+    for i, (x, wp, sw, bias) in enumerate(problems):
+        ldx = _rowmajor(x, "X")
+        ldp = _rowmajor(wp, "Wp")
+        m, k = x.shape
+        n = wp.shape[0]
+        y, ldy = _out_tensor(None, m, n, out, x.device)
+        ys.append(y)
+        arr[i] = Problem(x.data_ptr(), wp.data_ptr(), sw.data_ptr(), None if bias is None else bias.data_ptr(),
+                         y.data_ptr(), m, k, ldx, ldp, n, ldy)
+    flags = (RELU if relu else 0) | _OUT[out] | (STATIC_WEIGHTS if static_weights else 0)
+    _check(lib.w4a8_linear_grouped(arr, len(problems), flags, _stream(stream)), "w4a8_linear_grouped")
+    return ys
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
