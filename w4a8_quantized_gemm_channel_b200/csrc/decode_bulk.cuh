@@ -432,8 +432,8 @@ k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ld
 // ---------------------------------------------------------------------------
 // Grouped decode: many independent few-row linears in one persistent launch.
 // The problems' 16-channel groups are numbered one after another; block b
-// takes the contiguous run [T b / grid, T (b + 1) / grid) of the T groups, so
-// it switches problems rarely. Its producer streams every (group, stage) of
+// takes a contiguous run of them holding 1 / grid of all weight bytes, so it
+// switches problems rarely and the blocks finish together. Its producer streams every (group, stage) of
 // that run through one ring (slots of the largest stage, 16 x 2048 bytes)
 // with each problem's own tensor map; its consumers quantize a problem's
 // activation rows into shared memory (two passes over X, the arithmetic of
@@ -452,12 +452,29 @@ struct GroupedProblem {
     const float *bias;
     void *Y;
     int M, K, ldx, ldy, N, vec4, group0, pad;
+    long long bytes0;     // packed weight bytes of all earlier problems' groups
+    long long group_bytes;  // packed weight bytes of one of this problem's groups
 };
 struct GroupedTable {
     GroupedProblem p[MAX_GROUPED];
     int count;
     int total_groups;
+    long long total_bytes;
 };
+
+// The first group whose weights start at or after byte `b` of the run of all
+// groups (blocks split the work by weight bytes, not by group count: a group
+// of a long-K layer carries several times the bytes of a short one).
+__device__ __forceinline__ int grouped_first_group(const GroupedTable &tab, long long b) {
+    int p = 0;
+    while (p + 1 < tab.count && tab.p[p + 1].bytes0 <= b) ++p;
+    const GroupedProblem &q = tab.p[p];
+    const long long off = b - q.bytes0;
+    const int ng = (q.N + ROWS - 1) / ROWS;
+    int j = (int)((off + q.group_bytes - 1) / q.group_bytes);
+    if (j > ng) j = ng;
+    return q.group0 + j;
+}
 static_assert(sizeof(GroupedTable) <= 30 * 1024, "kernel parameter space");
 
 // Position in a block's run of (group, stage) items.
@@ -486,9 +503,10 @@ k_decode_grouped(const __grid_constant__ GroupedTable tab, unsigned flags, int r
     uint8_t *ring = dyn_smem;  // [ring_n][GROUPED_SLOT]
     int8_t *xs = reinterpret_cast<int8_t *>(dyn_smem + (size_t)ring_n * GROUPED_SLOT);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int T = tab.total_groups;
-    const int g_begin = (int)((long long)T * blockIdx.x / gridDim.x);
-    const int g_end = (int)((long long)T * (blockIdx.x + 1) / gridDim.x);
+    const long long B = tab.total_bytes;
+    const int g_begin = grouped_first_group(tab, B * blockIdx.x / gridDim.x);
+    const int g_end = blockIdx.x + 1 == gridDim.x ? tab.total_groups
+                                                    : grouped_first_group(tab, B * (blockIdx.x + 1) / gridDim.x);
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {

@@ -321,6 +321,7 @@ w4a8_status launch_grouped_chunk(const w4a8_problem *probs, int count, unsigned 
     std::lock_guard<std::mutex> lock(mu);
     memset(&tab, 0, sizeof(tab));
     int total = 0, max_m = 0, max_pitch = 0;
+    long long total_bytes = 0;
     for (int i = 0; i < count; ++i) {
         const w4a8_problem &p = probs[i];
         const dbulk::Geometry geo(p.K);
@@ -339,12 +340,16 @@ w4a8_status launch_grouped_chunk(const w4a8_problem *probs, int count, unsigned 
         q.N = p.N;
         q.vec4 = aligned16(p.X) && (p.ldx % 4 == 0);
         q.group0 = total;
+        q.bytes0 = total_bytes;
+        q.group_bytes = (long long)dbulk::ROWS * geo.kp;
         total += (p.N + dbulk::ROWS - 1) / dbulk::ROWS;
+        total_bytes += q.group_bytes * ((p.N + dbulk::ROWS - 1) / dbulk::ROWS);
         max_m = max_m > p.M ? max_m : p.M;
         max_pitch = max_pitch > geo.pitch ? max_pitch : geo.pitch;
     }
     tab.count = count;
     tab.total_groups = total;
+    tab.total_bytes = total_bytes;
     const int r = fq_rows(max_m);
     const long long xs = (long long)r * max_pitch;
     const long long ring = ((long long)dbulk::SMEM_BUDGET - xs) / dbulk::GROUPED_SLOT;
