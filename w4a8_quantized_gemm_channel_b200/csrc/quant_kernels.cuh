@@ -75,33 +75,28 @@ __device__ __forceinline__ float weight_scale_from_amax(unsigned bits) {
     return a == 0.0f ? 1.0f : __fdiv_rn(7.0f, a);
 }
 
-// Four codes (one per byte of w, each in [-8, 7]) -> 16 bits of nibbles,
-// the code of byte 0 in the lowest nibble.
-__device__ __forceinline__ uint32_t pack4_nibbles(uint32_t w) {
-    uint32_t x = w & 0x0F0F0F0Fu;
-    uint32_t y = (x | (x >> 4)) & 0x00FF00FFu;
-    return (y | (y >> 8)) & 0xFFFFu;
-}
-
 // ---------------------------------------------------------------------------
 // Weight pass 2: quantize and pack a tile of 64 k x (32 * VEC) output
-// channels. Reads are row-coalesced (float4 per lane for VEC = 4); codes are
-// transposed through shared memory so each output channel's 32 bytes of
-// packed nibbles leave as two 16-byte stores. Tiles cover k in [0, 2*ldp),
-// so every byte of every packed row (pad bytes included) is written.
-// grid = (ceil(N / (32 * VEC)), ceil(2*ldp / 64)), block = 256.
+// channels. Warp w reads the 8 consecutive rows k0 + 8w .. k0 + 8w + 7
+// (row-coalesced, float4 per lane for VEC = 4), so each thread holds 8
+// consecutive codes of each of its channels and packs them into one 32-bit
+// word in registers (code k0 + 8w + i in bits 4i..4i+3: even k in the low
+// nibble of its byte). The words go through shared memory as [warp][channel]
+// rows (16-byte stores, no bank conflicts); then each channel's four words
+// of one half-tile (32 codes) leave as one 16-byte store. Tiles cover k in
+// [0, 2*ldp), so every byte of every packed row (pad bytes included) is
+// written. grid = (ceil(N / (32 * VEC)), ceil(2*ldp / 64)), block = 256.
 // ---------------------------------------------------------------------------
 template <int VEC>
 __global__ void __launch_bounds__(256)
 k_quant_pack(const float *__restrict__ W, int K, int N, int ldw,
              const unsigned *__restrict__ amax_bits, uint8_t *__restrict__ Wp, int ldp) {
     constexpr int COLS = 32 * VEC;
-    constexpr int QS = 64 + 16;  // row pitch of the transposed codes (16-byte aligned)
-    __shared__ __align__(16) int8_t qs[COLS][QS];
+    __shared__ __align__(16) uint32_t pk[8][COLS];  // [warp][channel]: 8 codes of 8 consecutive k
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nb = blockIdx.x * COLS;
     const int n = nb + lane * VEC;
-    const int k0 = blockIdx.y * 64;
+    const int k0 = blockIdx.y * 64 + 8 * warp;
     float s[VEC];
 #pragma unroll
     for (int c = 0; c < VEC; ++c) s[c] = (n + c < N) ? weight_scale_from_amax(__ldg(amax_bits + n + c)) : 1.0f;
@@ -109,7 +104,7 @@ k_quant_pack(const float *__restrict__ W, int K, int N, int ldw,
     float v[8][VEC];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int k = k0 + warp + 8 * i;
+        const int k = k0 + i;
         if (k < K && n < N) {
             if constexpr (VEC == 4) {
                 const float4 f = __ldg(reinterpret_cast<const float4 *>(W + (size_t)k * ldw + n));
@@ -122,27 +117,30 @@ k_quant_pack(const float *__restrict__ W, int K, int N, int ldw,
             for (int c = 0; c < VEC; ++c) v[i][c] = 0.0f;
         }
     }
+    uint32_t word[VEC];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int c = 0; c < VEC; ++c) {
+        word[c] = 0;
 #pragma unroll
-        for (int c = 0; c < VEC; ++c)
-            qs[lane * VEC + c][warp + 8 * i] = (int8_t)clampi(__float2int_rn(__fmul_rn(v[i][c], s[c])), -8, 7);
-    __syncthreads();
-    // 2 threads per output channel row, 16 packed bytes (32 codes) each.
-    for (int tt = threadIdx.x; tt < 2 * COLS; tt += 256) {
-        const int r = tt >> 1, h = tt & 1;
-        const int nn = nb + r;
-        const int byte0 = k0 / 2 + 16 * h;  // a multiple of 16, as is ldp
-        if (nn < N && byte0 < ldp) {
-            const uint4 a = *reinterpret_cast<const uint4 *>(&qs[r][32 * h]);
-            const uint4 b = *reinterpret_cast<const uint4 *>(&qs[r][32 * h + 16]);
-            uint4 o;
-            o.x = pack4_nibbles(a.x) | (pack4_nibbles(a.y) << 16);
-            o.y = pack4_nibbles(a.z) | (pack4_nibbles(a.w) << 16);
-            o.z = pack4_nibbles(b.x) | (pack4_nibbles(b.y) << 16);
-            o.w = pack4_nibbles(b.z) | (pack4_nibbles(b.w) << 16);
-            *reinterpret_cast<uint4 *>(Wp + (size_t)nn * ldp + byte0) = o;
+        for (int i = 0; i < 8; ++i) {
+            const int q = clampi(__float2int_rn(__fmul_rn(v[i][c], s[c])), -8, 7);
+            word[c] |= ((uint32_t)q & 0xFu) << (4 * i);
         }
+    }
+    if constexpr (VEC == 4)
+        *reinterpret_cast<uint4 *>(&pk[warp][lane * 4]) = make_uint4(word[0], word[1], word[2], word[3]);
+    else
+        pk[warp][lane] = word[0];
+    __syncthreads();
+    // thread (h, r): channel nb + r, half-tile h = k in [32h, 32h + 32) = the
+    // words of warps 4h .. 4h + 3 = 16 packed bytes at byte k_tile/2 + 16h
+    for (int tt = threadIdx.x; tt < 2 * COLS; tt += 256) {
+        const int r = tt % COLS, h = tt / COLS;
+        const int nn = nb + r;
+        const int byte0 = blockIdx.y * 32 + 16 * h;  // a multiple of 16, as is ldp
+        if (nn < N && byte0 < ldp)
+            *reinterpret_cast<uint4 *>(Wp + (size_t)nn * ldp + byte0) =
+                make_uint4(pk[4 * h][r], pk[4 * h + 1][r], pk[4 * h + 2][r], pk[4 * h + 3][r]);
     }
 }
 
