@@ -36,9 +36,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "W4A8 linear: TOPS (prefill) and HBM GB/s (decode) vs B200 roofline"
-# DRAM bytes (read + write) of one k_decode_ring launch at M = 1, K = N = 4096, from the ncu capture
-# summarized in profiles/k_decode_ring_m1_k4096_n4096.md; recapture when the kernel changes.
-RING_TRAFFIC_PER_LAUNCH = 8433920
+# DRAM bytes (read + write) per launch of the decode product kernels at K = N = 4096, by kernel, from
+# the ncu captures summarized in profiles/ (k_decode_ring at M = 1; k_linear_decode: mean of its M = 4 and
+# M = 16 launches); recapture when a kernel changes.
+DECODE_TRAFFIC_PER_LAUNCH = {"k_decode_ring": 8433920, "k_linear_decode": 8460480}
+DECODE_TRAFFIC_NOTE = {
+    "k_decode_ring": "profiles/k_decode_ring_m1_k4096_n4096.md (M=1)",
+    "k_linear_decode": "profiles/launches_decode_bench_k4096_n4096.md (mean of M=4 and M=16)",
+}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
@@ -294,7 +299,8 @@ def time_steps(torch, wl, steps, warmup, dist=None):
 def time_kernel_only(torch, nat, wl):
     """Average device time per decode-kernel launch (w4a8_linear_q, INT8
     activations already quantized) in a back-to-back graph over the rotating
-    weight pool, per M; returns {m: (ms_per_launch, algorithmic_bytes)}."""
+    weight pool, per M; returns {m: (ms_per_launch, algorithmic_bytes,
+    kernel_name)}."""
     out = {}
     ldp = nat.packed_ld(wl.K)
     for m in wl.MS:
@@ -304,6 +310,8 @@ def time_kernel_only(torch, nat, wl):
         def run():
             for i in range(reps):
                 nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], y=wl.y[m], static_weights=True)
+        nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[0], wl.sw[0], y=wl.y[m], static_weights=True)
+        kernel = nat.last_kernel()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
@@ -324,7 +332,7 @@ def time_kernel_only(torch, nat, wl):
         torch.cuda.synchronize()
         ms = start.elapsed_time(stop) / (n_rep * reps)
         nbytes = wl.N * ldp + 4 * wl.N + m * xq.shape[1] + 4 * m + 4 * m * wl.N
-        out[m] = (ms, nbytes)
+        out[m] = (ms, nbytes, kernel)
     return out
 
 
@@ -724,10 +732,14 @@ def main():
     value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9
 
     kern = time_kernel_only(torch, native, wl)
-    # the dominant kernel (k_decode_ring: 60 % of the launch list) serves M <= 8
-    ring_ms = [m for m in kern if m <= 8]
-    k_ms = sum(kern[m][0] for m in ring_ms)
-    k_bytes = sum(kern[m][1] for m in ring_ms)
+    # the dominant product kernel: the one with the most device time over the step's M
+    by_kernel = {}
+    for m, (t_ms, nbytes, name) in kern.items():
+        by_kernel.setdefault(name, []).append(m)
+    dom = max(by_kernel, key=lambda name: sum(kern[m][0] for m in by_kernel[name]))
+    dom_ms = by_kernel[dom]
+    k_ms = sum(kern[m][0] for m in dom_ms)
+    k_bytes = sum(kern[m][1] for m in dom_ms)
     peaks, peak_kind = measured_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     achieved = k_bytes / (k_ms * 1e-3) / 1e9
@@ -743,13 +755,12 @@ def main():
         "data": "synthetic", "config": wl.config(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": RING_TRAFFIC_PER_LAUNCH,
-                     "traffic_note": "dram bytes read+written per k_decode_ring launch (M=1), ncu capture "
-                                     "in profiles/k_decode_ring_m1_k4096_n4096.md",
-                     "kernel": f"k_decode_ring over M in {ring_ms} (w4a8_linear_q back-to-back over "
-                               "rotating weights, static-weights promise); per_m also lists "
-                               "k_linear_decode at M = 16",
-                     "per_m": {str(m): {"us": round(v[0] * 1e3, 3), "bytes": v[1],
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": DECODE_TRAFFIC_PER_LAUNCH.get(dom),
+                     "traffic_note": f"dram bytes read+written per {dom} launch, ncu capture in "
+                                     f"{DECODE_TRAFFIC_NOTE.get(dom, '(none)')}",
+                     "kernel": f"{dom} over M in {dom_ms} (w4a8_linear_q back-to-back over rotating "
+                               "weights, static-weights promise); per_m lists every M's kernel",
+                     "per_m": {str(m): {"kernel": v[2], "us": round(v[0] * 1e3, 3), "bytes": v[1],
                                         "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
                                for m, v in kern.items()}},
         "stages": {"quantize_pack": {"ms": round(qp_ms, 4), "bytes": qp_bytes,

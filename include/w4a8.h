@@ -221,6 +221,14 @@ W4A8_API unsigned w4a8_last_path(void);
  * if that call had M == 0). */
 W4A8_API unsigned w4a8_last_launch_count(void);
 
+/* Name of the product kernel that the calling thread's last successful
+ * w4a8_linear / w4a8_linear_q / w4a8_linear_noalloc / w4a8_linear_grouped
+ * call enqueued ("k_decode_ring", "k_linear_decode", "k_gemm_tc",
+ * "k_linear_generic" or "k_decode_grouped"), not counting the activation
+ * pass; "" if none, or if that call had nothing to do. A static string that
+ * the caller must not free. */
+W4A8_API const char *w4a8_last_kernel(void);
+
 /*
  * w4a8_selftest_timeout - exercises the library's failure path without
  * faulting the GPU. Every wait inside the kernels is bounded: after about a

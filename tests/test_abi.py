@@ -104,10 +104,10 @@ def test_last_launch_count_starts_at_zero_per_thread():
     import threading
     from w4a8_quantized_gemm_channel_b200 import native
     seen = []
-    t = threading.Thread(target=lambda: seen.append(native.last_launch_count()))
+    t = threading.Thread(target=lambda: seen.append((native.last_launch_count(), native.last_kernel())))
     t.start()
     t.join()
-    assert seen == [0]
+    assert seen == [(0, "")]
 
 
 def test_selftest_timeout_rejects_bad_limits():

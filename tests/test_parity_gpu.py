@@ -237,6 +237,27 @@ def test_decode_full_size(nat, m):
     assert np.array_equal(host(acc), oracle.linear(c.x, wp, sw, synth.DECODE_K, out="s32"))
 
 
+@pytest.mark.parametrize("m,k,groups_over_2sm,kernel", [
+    (1, 4096, -40, "k_decode_ring"), (2, 4096, -40, "k_decode_ring"), (3, 4096, -40, "k_linear_decode"),
+    (8, 4096, -290, "k_linear_decode"), (8, 4097, -290, "k_decode_ring"), (8, 4096, 0, "k_linear_decode"),
+    (8, 4096, 1, "k_decode_ring"), (16, 4096, -40, "k_linear_decode")])
+def test_decode_kernel_choice_and_bits(nat, m, k, groups_over_2sm, kernel):
+    """Few-row products with INT8 input on both sides of the rule that hands
+    short layers (at most two 16-channel groups per SM) with K <= 4096 and
+    M >= 3 to the register-path kernel: the kernel named, and the INT32
+    accumulators bit for bit, with and without the static-weights promise."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n = 16 * (2 * sms + groups_over_2sm)
+    x, w, _ = _case(m, k, n, seed=1300 + m + k)
+    wp, sw = oracle.w4_quantize_pack(w)
+    ref = oracle.linear(x, wp, sw, k, out="s32")
+    xq, sx = nat.a8_quantize_rows(dev(x))
+    for static in (False, True):
+        acc = nat.w4a8_linear_q(xq, sx, k, dev(wp), dev(sw), out="s32", static_weights=static)
+        assert nat.last_kernel() == kernel
+        assert np.array_equal(host(acc), ref)
+
+
 def _sampled_check(nat, x, w, wpd, swd, rows, cols, relu=False, path="auto"):
     """Full-size run on the GPU; the oracle recomputes sampled rows x channels
     (each sampled row is quantized over its full K)."""

@@ -49,6 +49,7 @@ SIGNATURES = {
     "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_last_path": (_U, []),
     "w4a8_last_launch_count": (_U, []),
+    "w4a8_last_kernel": (ctypes.c_char_p, []),
     "w4a8_selftest_timeout": (_I, [ctypes.c_longlong, _P]),
     "w4a8_linear_grouped": (_I, [ctypes.POINTER(Problem), _I, _U, _P]),
     "w4a8_get_device_status": (_I, [_I, _P]),
@@ -240,6 +241,11 @@ def last_path() -> str:
 
 def last_launch_count() -> int:
     return lib.w4a8_last_launch_count()
+
+
+def last_kernel() -> str:
+    """Name of the product kernel of this thread's last call ("" if none)."""
+    return lib.w4a8_last_kernel().decode()
 
 
 def selftest_timeout(cycles: int = 1_000_000, stream=None):
