@@ -65,6 +65,8 @@ def _load():
                 "oracle_dequant": [P, I, I, I, P, P, P, I, P, I],
                 "oracle_f32_to_bf16_array": [P, ctypes.c_size_t, P],
                 "oracle_quantize_weight": [ctypes.c_float, ctypes.c_float],
+                "oracle_w8_quantize": [P, I, I, I, P, I, P],
+                "oracle_gemm8_s32": [P, I, I, I, P, I, I, P, I],
             }.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
@@ -208,6 +210,57 @@ def linear_q(xq: np.ndarray, sx: np.ndarray, wp: np.ndarray, sw: np.ndarray, k: 
              bias: np.ndarray | None = None, relu: bool = False, out: str = "f32"):
     """Steps 4-6 on already-quantized activations."""
     acc = gemm_s32(xq, k, wp)
+    if out == "s32":
+        return acc
+    y = dequant(acc, sx, sw, bias, relu)
+    return to_bf16_bits(y) if out == "bf16" else y
+
+
+# ----------------------------------------------------------------- W8A8 ---
+# The INT8 path that the page presents INT4 as an extension of: the same steps
+# with 8-bit weight codes (scale 127 / max|W[:,n]|, range [-127, 127]) stored
+# one per byte. Activation quantization and dequantization are steps 3 and 6
+# above, unchanged.
+
+def w8_ld(k: int) -> int:
+    """Bytes per INT8 weight row: K rounded up to 16."""
+    return (k + 15) // 16 * 16
+
+
+def w8_quantize(w: np.ndarray, ldw8: int | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """W[K][N] float32 -> (Q8[N][ldw8] int8 codes, pad 0; sw[N] float32)."""
+    w = _f32(w)
+    k, n = w.shape
+    ldw8 = w8_ld(k) if ldw8 is None else ldw8
+    q8 = np.empty((n, ldw8), np.int8)
+    sw = np.empty(n, np.float32)
+    _check(_load().oracle_w8_quantize(_ptr(w), k, n, n, _ptr(q8), ldw8, _ptr(sw)), "w8_quantize")
+    return q8, sw
+
+
+def gemm8_s32(xq: np.ndarray, k: int, q8: np.ndarray) -> np.ndarray:
+    """acc[M][N] = sum_k xq[m][k] * q8[n][k] (exact, must fit INT32)."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    q8 = np.ascontiguousarray(q8, dtype=np.int8)
+    m, ldq = xq.shape
+    n, ldw8 = q8.shape
+    acc = np.empty((m, n), np.int32)
+    _check(_load().oracle_gemm8_s32(_ptr(xq), m, k, ldq, _ptr(q8), n, ldw8, _ptr(acc), n),
+           "gemm8_s32")
+    return acc
+
+
+def linear8(x: np.ndarray, q8: np.ndarray, sw: np.ndarray, k: int,
+            bias: np.ndarray | None = None, relu: bool = False, out: str = "f32"):
+    """One W8A8 Dense layer on float32 input (steps 3, 5, 6)."""
+    xq, sx = a8_quantize_rows(x)
+    return linear8_q(xq, sx, q8, sw, k, bias=bias, relu=relu, out=out)
+
+
+def linear8_q(xq: np.ndarray, sx: np.ndarray, q8: np.ndarray, sw: np.ndarray, k: int,
+              bias: np.ndarray | None = None, relu: bool = False, out: str = "f32"):
+    """W8A8 steps 5-6 on already-quantized activations."""
+    acc = gemm8_s32(xq, k, q8)
     if out == "s32":
         return acc
     y = dequant(acc, sx, sw, bias, relu)

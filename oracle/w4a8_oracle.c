@@ -21,6 +21,13 @@
  * sx = 127 / max|X[m,:]| (1 for an all-zero row), INT8 clamp [-127, 127];
  * dequantization y = float(acc) / (sx * sw).
  *
+ * W8A8 (the INT8 path that the same page says INT4 extends, section "How it
+ * works", closing paragraph): steps 1-6 with 8-bit weights and no packing.
+ * The page names that path without its constants; read here as the INT4
+ * path's arithmetic with the 8-bit symmetric range of its own activation
+ * step: sw = 127 / max|W[:,n]| (1 for a zero column), q = clamp(rne(w * sw),
+ * -127, 127), one byte per code, rows of ldw8 >= K bytes with zero pad.
+ *
  * Precision: the page's model is float32 end to end (its inputs are cast with
  * astype("float32")), and float32 decides every integer code, so each step
  * below runs in float32 with IEEE round-to-nearest. Build flags:
@@ -253,4 +260,50 @@ int oracle_linear(const float *X, int M, int K, int ldx,
     rc = oracle_gemm_s32(Xq, M, K, K, Wp, N, ldp, acc, N);
     if (rc) return rc;
     return oracle_dequant(acc, M, N, N, sx, sw, bias, relu, Y, ldy);
+}
+
+/* ---------------------------------------------------------------------------
+ * W8A8, steps 1-2: per-output-channel scale sw[n] = 127 / max_k |W[k][n]|
+ * (1 for an all-zero column) and codes q = clamp(rne(w * sw), -127, 127),
+ * stored one per byte: Q8[N][ldw8], bytes k >= K of each row 0.
+ * ------------------------------------------------------------------------- */
+int oracle_w8_quantize(const float *W, int K, int N, int ldw, int8_t *Q8, int ldw8, float *sw)
+{
+    if (!W || !Q8 || !sw || K < 1 || N < 1 || ldw < N || ldw8 < K) return ORACLE_BAD_ARG;
+    for (int n = 0; n < N; ++n) {
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(W[(size_t)k * ldw + n]);
+            if (a > amax) amax = a;
+        }
+        sw[n] = (amax == 0.0f) ? 1.0f : 127.0f / amax;
+        int8_t *row = Q8 + (size_t)n * ldw8;
+        memset(row, 0, (size_t)ldw8);
+        for (int k = 0; k < K; ++k) {
+            float t = W[(size_t)k * ldw + n] * sw[n];
+            row[k] = (int8_t)clamp_int((int)round_half_even(t), -127, 127);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* W8A8, step 5: acc[m][n] = sum_k xq[m][k] * q8[n][k], exact (int64) and
+ * required to fit INT32. */
+int oracle_gemm8_s32(const int8_t *Xq, int M, int K, int ldq,
+                     const int8_t *Q8, int N, int ldw8,
+                     int32_t *acc, int ldacc)
+{
+    if (M < 0 || K < 1 || N < 1 || ldq < K || ldw8 < K || ldacc < N) return ORACLE_BAD_ARG;
+    if (M == 0) return ORACLE_OK;
+    if (!Xq || !Q8 || !acc) return ORACLE_BAD_ARG;
+    for (int m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            int64_t s = 0;
+            for (int k = 0; k < K; ++k)
+                s += (int64_t)Xq[(size_t)m * ldq + k] * (int64_t)Q8[(size_t)n * ldw8 + k];
+            if (s > INT32_MAX || s < INT32_MIN) return ORACLE_OVERFLOW;
+            acc[(size_t)m * ldacc + n] = (int32_t)s;
+        }
+    }
+    return ORACLE_OK;
 }

@@ -306,3 +306,117 @@ def test_minimal_model_is_deterministic():
     a = oracle.mlp(d.x, d.w1, d.b1, d.w2, d.b2)
     b = oracle.mlp(d.x, d.w1, d.b1, d.w2, d.b2)
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+# ------------------------------------------------------------------ W8A8 ---
+# The INT8 path the page presents INT4 as an extension of (section "How it
+# works", closing paragraph): 8-bit codes, scale 127 / abs-max, no packing.
+
+def test_w8_codes_hand_worked():
+    """Abs-max 1 gives sw = 127; 0.5 * 127 = 63.5 is a tie and rounds to the
+    even 64 (-63.5 to -64), 0.25 * 127 = 31.75 rounds to 32, and the abs-max
+    element maps to 127. Pad bytes past K are 0."""
+    w = np.array([[1.0], [-0.5], [0.25], [0.5], [-1.0]], np.float32)
+    q8, sw = oracle.w8_quantize(w, ldw8=16)
+    assert sw.tolist() == [127.0]
+    assert q8[0, :5].tolist() == [127, -64, 32, 64, -127]
+    assert not q8[0, 5:].any()
+
+
+def test_w8_codes_range_extremes_and_scale():
+    """Codes stay in [-127, 127]; the element attaining a column's abs-max maps
+    to exactly +-127; the scale is 127 / abs-max in float32."""
+    w = _random_w(k=300, n=40, seed=31)
+    q8, sw = oracle.w8_quantize(w)
+    assert q8.min() >= -127 and q8.max() <= 127
+    for n in range(w.shape[1]):
+        kmax = int(np.argmax(np.abs(w[:, n])))
+        assert q8[n, kmax] == (127 if w[kmax, n] > 0 else -127)
+    amax = np.abs(w).max(axis=0)
+    assert np.array_equal(sw, (np.float32(127.0) / amax).astype(np.float32))
+
+
+def test_w8_invariances_and_zero_column():
+    """Powers of two leave the codes unchanged and divide the scale exactly;
+    negating W negates the codes; an all-zero column has scale 1, codes 0."""
+    w = _random_w(k=200, n=8, seed=32)
+    w[:, 5] = 0.0
+    q0, sw0 = oracle.w8_quantize(w)
+    assert sw0[5] == np.float32(1.0) and not q0[5].any()
+    for j in (-4, 3):
+        qj, swj = oracle.w8_quantize((w * np.float32(2.0 ** j)).astype(np.float32))
+        assert np.array_equal(qj, q0)
+        nz = np.arange(w.shape[1]) != 5  # the zero column keeps scale 1
+        assert np.array_equal((swj * np.float32(2.0 ** j))[nz], sw0[nz]) and swj[5] == 1.0
+    q1, sw1 = oracle.w8_quantize(-w)
+    assert np.array_equal(sw1, sw0) and np.array_equal(q1, -q0)
+
+
+def test_w8_weight_error_bound():
+    """|w - q/sw| <= 0.5/sw everywhere: the abs-max maps to 127, nothing clips."""
+    w = _random_w(k=512, n=64, seed=33).astype(np.float64)
+    q8, sw = oracle.w8_quantize(w.astype(np.float32))
+    err = np.abs(w.T - q8[:, :512].astype(np.float64) / sw.astype(np.float64)[:, None])
+    assert (err <= 0.5 / sw.astype(np.float64)[:, None] * (1 + 1e-6)).all()
+
+
+def test_gemm8_matches_float64_matmul():
+    """Integer products summed in float64 are exact while |acc| < 2^53; the
+    codes span the full INT8 range on both sides, pad bytes are ignored."""
+    rng = synth.rng_for(34, 0)
+    for (m, k, n) in ((1, 1, 1), (3, 7, 5), (24, 777, 40)):
+        q8 = np.zeros((n, (k + 15) // 16 * 16), np.int8)
+        q8[:, :k] = rng.integers(-127, 128, size=(n, k))
+        q8[:, k:] = 99  # pad bytes: must not be read
+        xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+        acc = oracle.gemm8_s32(xq, k, q8)
+        ref = xq.astype(np.float64) @ q8[:, :k].astype(np.float64).T
+        assert np.array_equal(acc.astype(np.float64), ref)
+
+
+def test_gemm8_int32_overflow_is_reported():
+    k = 133_200  # 127 * 127 * k > 2^31 - 1
+    xq = np.full((1, k), 127, np.int8)
+    q8 = np.full((1, k), 127, np.int8)
+    with pytest.raises(oracle.OracleError):
+        oracle.gemm8_s32(xq, k, q8)
+    k = 133_144  # the largest K whose worst case fits
+    assert oracle.gemm8_s32(xq[:, :k], k, q8[:, :k])[0, 0] == 127 * 127 * k
+
+
+def test_linear8_exact_when_codes_are_exact():
+    """Abs-maxes 63.5 (X) and 63.5 (W) give sx = sw = 2; every value is a
+    half-integer, so y = acc / 4 equals X @ W exactly (a swapped or dropped
+    scale misses by a factor of 4 or 16)."""
+    rng = synth.rng_for(35, 0)
+    m, k, n = 5, 60, 7
+    wq = rng.integers(-127, 128, size=(k, n)).astype(np.float32)
+    wq[0, :] = 127
+    xq = rng.integers(-127, 128, size=(m, k)).astype(np.float32)
+    xq[:, 0] = -127
+    w, x = wq / 2, xq / 2
+    q8, sw = oracle.w8_quantize(w)
+    assert (sw == 2.0).all()
+    y = oracle.linear8(x, q8, sw, k)
+    assert np.array_equal(y.astype(np.float64), x.astype(np.float64) @ w.astype(np.float64))
+
+
+def test_linear8_error_bound_and_tighter_than_int4():
+    """The same error bound as the INT4 layer with e_w = 0.5/sw, sw = 127 /
+    abs-max; on the same data the INT8 weights' error is well below INT4's."""
+    x, _ = synth.linear_activations(8, 640, seed=36, outlier_count=3, outlier_factor=20.0)
+    w = synth.linear_weights(640, 48, 0.02, seed=36)
+    q8, sw = oracle.w8_quantize(w)
+    xq, sx = oracle.a8_quantize_rows(x)
+    y8 = oracle.linear8(x, q8, sw, 640)
+    x64, w64 = x.astype(np.float64), w.astype(np.float64)
+    exact = x64 @ w64
+    ew = 0.5 / sw.astype(np.float64)
+    ex = 0.5 / sx.astype(np.float64)
+    bound = (np.abs(x64).sum(1)[:, None] * ew[None, :] + ex[:, None] * np.abs(w64).sum(0)[None, :]
+             + 640 * ex[:, None] * ew[None, :])
+    slack = 1e-5 * (np.abs(x64) @ np.abs(w64)) + 1e-6
+    assert (np.abs(y8 - exact) <= bound + slack).all()
+    wp, sw4 = oracle.w4_quantize_pack(w)
+    y4 = oracle.linear(x, wp, sw4, 640)
+    assert np.abs(y8 - exact).mean() < 0.5 * np.abs(y4 - exact).mean()
