@@ -85,6 +85,10 @@ enum {
 /* Largest K whose INT32 accumulator cannot overflow: 127 * 8 * K < 2^31. */
 #define W4A8_MAX_K 2097152
 
+/* Largest K for the W8A8 path: 127 * 127 * K < 2^31 keeps the INT32
+ * accumulator exact for any codes. */
+#define W8A8_MAX_K 133144
+
 /* Bytes per packed output-channel row: ceil(K/2) rounded up to a multiple of
  * 16 (the stride every tensor-core tile load needs). Returns -1 if K < 1. */
 W4A8_API int w4a8_packed_ld(int K);
@@ -211,6 +215,56 @@ typedef struct w4a8_problem {
 } w4a8_problem;
 
 W4A8_API w4a8_status w4a8_linear_grouped(const w4a8_problem *probs, int count, unsigned flags, void *stream);
+
+/*
+ * W8A8 - the INT8 path that the guide's INT4 scheme extends ("How it works",
+ * closing paragraph: the INT4 path is the INT8 path plus an unpack). Read as
+ * the same steps with one 8-bit weight code per byte:
+ *   weights - sw = 127 / max|W[:,n]| (1 for an all-zero column),
+ *             q = clamp(rne(w * sw), -127, 127), rows of ldw8 bytes;
+ *   activations, product and output - as for w4a8_linear (steps 3, 5, 6).
+ * Kernels: decode for M <= 16, the tcgen05 GEMM otherwise (the weight tile
+ * goes to the tensor cores as it is, no unpack), the generic kernel for tiny
+ * problems; the W4A8_PATH_* flags force one as for the INT4 layer.
+ */
+
+/* Bytes per INT8 weight row: K rounded up to a multiple of 16 (-1 if K < 1). */
+W4A8_API int w8a8_ld(int K);
+
+/*
+ * w8_quantize - W8A8 steps 1-2.
+ *   W   [K][ldw] float32 (the Keras kernel layout), ldw >= N, finite.
+ *   Wq  [N][ldw8] int8 out, ldw8 >= K and a multiple of 16, 16-byte aligned;
+ *       bytes K..ldw8-1 of every row are written 0.
+ *   sw  [N] float32 out: 127 / max_k |W[k][n]|, or 1 for an all-zero column.
+ * Requires 1 <= K <= W8A8_MAX_K, N >= 1. Uses sw as scratch while it runs.
+ */
+W4A8_API w4a8_status w8_quantize(const float *W, int K, int N, int ldw,
+                        int8_t *Wq, int ldw8, float *sw, void *stream);
+
+/*
+ * w8a8_linear - W8A8 steps 3, 5, 6 on float32 activations: quantize each row
+ * of X to INT8 (into the workspace), multiply with the INT8 weights,
+ * accumulate in INT32, dequantize, add the bias, apply ReLU. Arguments,
+ * flags, workspace and errors as for w4a8_linear, with Wq/ldw8 as produced by
+ * w8_quantize (bytes K..round_up(K,16)-1 of each row must be 0; bytes past
+ * that are never read) and 1 <= K <= W8A8_MAX_K. Always two launches: the
+ * activation pass, then the product.
+ */
+W4A8_API w4a8_status w8a8_linear(const float *X, int M, int K, int ldx,
+                        const int8_t *Wq, int ldw8, const float *sw, int N,
+                        const float *bias, unsigned flags,
+                        void *Y, int ldy,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w8a8_linear_q - steps 5-6 on INT8 activations Xq [M][ldq] (ldq >= K, a
+ * multiple of 16, 16-byte aligned) with scales sx [M], natural k order.
+ * Other arguments as for w8a8_linear; no workspace.
+ */
+W4A8_API w4a8_status w8a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                          const int8_t *Wq, int ldw8, const float *sw, int N,
+                          const float *bias, unsigned flags, void *Y, int ldy, void *stream);
 
 /* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
  * last successful w4a8_linear / w4a8_linear_q call enqueued; 0 if none. */

@@ -92,6 +92,46 @@ def test_quantize_argument_checks():
     assert lib.w4a8_linear_q(24, 2, 64, 64, 64, 4096, 32, 64, 8, None, 0, 8192, 8, None) == 1  # Xq misaligned
 
 
+def _linear8(lib, **kw):
+    a = dict(X=16, M=4, K=64, ldx=64, Wq=4096, ldw8=64, sw=8192, N=8, bias=None, flags=0,
+             Y=12288, ldy=8, ws=16384, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return lib.w8a8_linear(a["X"], a["M"], a["K"], a["ldx"], a["Wq"], a["ldw8"], a["sw"], a["N"],
+                           a["bias"], a["flags"], a["Y"], a["ldy"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(K=0), 1), (dict(N=0), 1), (dict(M=-1), 1),
+    (dict(K=133145, ldx=133145, ldw8=133152), 1),  # past W8A8_MAX_K
+    (dict(ldw8=48), 1),           # ldw8 < K
+    (dict(ldw8=72), 1),           # not a multiple of 16
+    (dict(Wq=4100), 1),           # Wq not 16-byte aligned
+    (dict(ldx=63), 1), (dict(ldy=7), 1), (dict(Y=None), 1), (dict(sw=None), 1),
+    (dict(flags=0x04 | 0x01), 1), (dict(flags=0x100), 1),
+    (dict(ws=None), 3), (dict(wsb=10), 3),
+    (dict(M=0), 0),
+])
+def test_w8a8_argument_checks(kw, want):
+    """The W8A8 calls reject bad arguments before any device work."""
+    from w4a8_quantized_gemm_channel_b200 import native
+    assert _linear8(native.lib, **kw) == want
+
+
+def test_w8a8_sizes_and_quantize_checks():
+    from w4a8_quantized_gemm_channel_b200 import native
+    import oracle
+    for k in (1, 15, 16, 17, 4096, 28672):
+        assert native.w8a8_ld(k) == oracle.w8_ld(k)
+    assert native.w8a8_ld(0) == -1
+    lib = native.lib
+    assert lib.w8_quantize(16, 0, 8, 8, 4096, 16, 64, None) == 1          # K = 0
+    assert lib.w8_quantize(16, 64, 8, 7, 4096, 64, 64, None) == 1         # ldw < N
+    assert lib.w8_quantize(16, 64, 8, 8, 4096, 48, 64, None) == 1         # ldw8 < K
+    assert lib.w8_quantize(16, 64, 8, 8, 4104, 64, 64, None) == 1         # Wq misaligned
+    assert lib.w8a8_linear_q(16, 0, 64, 64, 64, 4096, 64, 64, 8, None, 0, 8192, 8, None) == 0  # M = 0
+    assert lib.w8a8_linear_q(24, 2, 64, 64, 64, 4096, 64, 64, 8, None, 0, 8192, 8, None) == 1  # Xq misaligned
+
+
 def test_no_device_means_unsupported_not_a_crash():
     import torch
     if torch.cuda.is_available():

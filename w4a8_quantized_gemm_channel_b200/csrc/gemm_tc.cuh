@@ -53,6 +53,12 @@ template <int BT> struct Ring;
 template <> struct Ring<192> { static constexpr int STAGES = 3, A_SLOTS = 2; };  // 3 x 64 KB, 384 + 128 cols
 template <> struct Ring<128> { static constexpr int STAGES = 4, A_SLOTS = 4; };  // 4 x 48 KB, 256 + 256 cols
 template <> struct Ring<64> { static constexpr int STAGES = 6, A_SLOTS = 4; };   // 6 x 32 KB, 128 + 256 cols
+// The W8A8 form: weight tiles of one byte per code are twice as large, so
+// fewer stages fit the same shared memory.
+template <int BT> struct Ring8;
+template <> struct Ring8<192> { static constexpr int STAGES = 2, A_SLOTS = 2; };  // 2 x 80 KB, 384 + 128 cols
+template <> struct Ring8<128> { static constexpr int STAGES = 3, A_SLOTS = 2; };  // 3 x 64 KB, 256 + 128 cols
+template <> struct Ring8<64> { static constexpr int STAGES = 4, A_SLOTS = 4; };   // 4 x 48 KB, 128 + 256 cols
 // Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
 // it % UNPACK_WG, so the groups overlap their shared-memory reads, integer
 // work and TMEM stores.
@@ -63,23 +69,6 @@ constexpr int FIRST_EPI_WARP = FIRST_UNPACK_WARP + 4 * UNPACK_WG;
 constexpr int NUM_THREADS = 32 * (FIRST_EPI_WARP + 4);
 constexpr int TMEM_COLS = 512;
 constexpr int A_COLS = BK / 4;     // TMEM columns per A slot (4 INT8 per column)
-constexpr int W_TILE_BYTES = BM * BK / 2;
-
-template <int BT>
-struct alignas(1024) Smem {
-    uint8_t act[Ring<BT>::STAGES][BT * BK];       // activation tiles: BK / XBOX boxes of [BT][128 B], 128B-swizzled
-    uint8_t wpk[Ring<BT>::STAGES][W_TILE_BYTES];  // packed weight tiles [BM][128 B], 128B-swizzled
-    uint64_t full[Ring<BT>::STAGES];              // TMA landed (tx-count barrier)
-    uint64_t empty[Ring<BT>::STAGES];             // MMAs reading the stage finished
-    uint64_t aready[Ring<BT>::A_SLOTS];           // A slot written to TMEM (4 unpack warps)
-    uint64_t acc_full[2];                // accumulator ready for the epilogue
-    uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
-    uint64_t mma_done;                   // final drain of the MMA pipe
-    float rsx[BT];                       // 1/sx of the epilogue's current token tile
-    float tsx[BT];                       // sx of the same tokens
-    uint32_t tmem_base;
-    int abort;
-};
 
 // How the weight warpgroups widen nibbles to the INT8 A operand.
 //  UNPACK_SEXT: sign-extend each nibble (byte = q), then restore k order with
@@ -92,8 +81,38 @@ struct alignas(1024) Smem {
 //  UNPACK_X16_PERM: as UNPACK_X16 without the byte permutes: the activations
 //      were stored with each group of 8 k reordered to k0 k2 k4 k6 k1 k3 k5 k7
 //      (see k_act_quant), which is the order the masks produce.
-enum { UNPACK_SEXT = 0, UNPACK_X16 = 1, UNPACK_X16_PERM = 2 };
+//  UNPACK_NONE: the W8A8 path - the weight tile already holds one INT8 code
+//      per byte (two 128-byte boxes per row and stage, like the
+//      activations), and the weight warps copy it into TMEM unchanged.
+enum { UNPACK_SEXT = 0, UNPACK_X16 = 1, UNPACK_X16_PERM = 2, UNPACK_NONE = 3 };
 constexpr int TC_X16_MAX_K = 131072;
+
+// Ring sizes and the weight tile of a kernel form.
+template <int BT, int UNPACK>
+struct Cfg {
+    static constexpr bool W8 = UNPACK == UNPACK_NONE;
+    static constexpr int STAGES = W8 ? Ring8<BT>::STAGES : Ring<BT>::STAGES;
+    static constexpr int A_SLOTS = W8 ? Ring8<BT>::A_SLOTS : Ring<BT>::A_SLOTS;
+    static constexpr int W_TILE_BYTES = W8 ? BM * BK : BM * BK / 2;
+    static constexpr int SHIFT = (UNPACK == UNPACK_X16 || UNPACK == UNPACK_X16_PERM) ? 4 : 0;
+};
+
+template <int BT, int UNPACK>
+struct alignas(1024) Smem {
+    using C = Cfg<BT, UNPACK>;
+    uint8_t act[C::STAGES][BT * BK];          // activation tiles: BK / XBOX boxes of [BT][128 B], 128B-swizzled
+    uint8_t wpk[C::STAGES][C::W_TILE_BYTES];  // weight tiles: [BM][128 B] packed, or W8: two boxes of [BM][128 B]
+    uint64_t full[C::STAGES];                 // TMA landed (tx-count barrier)
+    uint64_t empty[C::STAGES];                // MMAs reading the stage finished
+    uint64_t aready[C::A_SLOTS];              // A slot written to TMEM (4 unpack warps)
+    uint64_t acc_full[2];                // accumulator ready for the epilogue
+    uint64_t acc_empty[2];               // epilogue drained the accumulator (4 warps)
+    uint64_t mma_done;                   // final drain of the MMA pipe
+    float rsx[BT];                       // 1/sx of the epilogue's current token tile
+    float tsx[BT];                       // sx of the same tokens
+    uint32_t tmem_base;
+    int abort;
+};
 
 template <int BT>
 constexpr int d_col(int buf) { return buf * BT; }
@@ -151,8 +170,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
           int M, int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
           const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
-    constexpr int STAGES = Ring<BT>::STAGES;
-    constexpr int A_SLOTS = Ring<BT>::A_SLOTS;
+    constexpr int STAGES = Cfg<BT, UNPACK>::STAGES;
+    constexpr int A_SLOTS = Cfg<BT, UNPACK>::A_SLOTS;
+    constexpr int W_TILE_BYTES = Cfg<BT, UNPACK>::W_TILE_BYTES;
     static_assert(A_SLOTS % UNPACK_WG == 0, "each warpgroup owns fixed TMEM slots");
     // The unpack warps reuse A slot it % A_SLOTS once the stage barrier of
     // iteration it - A_SLOTS has flipped; that barrier is not reused before
@@ -161,7 +181,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
     static_assert(2 * BT + A_SLOTS * A_COLS <= TMEM_COLS, "TMEM budget");
     static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
     extern __shared__ uint8_t smem_raw[];
-    Smem<BT> &sm = *reinterpret_cast<Smem<BT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<BT, UNPACK> &sm = *reinterpret_cast<Smem<BT, UNPACK> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_kb = (K + BK - 1) / BK;
     const int tiles_m = (M + BT - 1) / BT;
@@ -212,7 +232,14 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!ptx::mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&sm.full[stage], BT * BK + W_TILE_BYTES);
-                    ptx::tma_load_2d(sm.wpk[stage], &tm_w, kb * (BK / 2), n_tile * BM, &sm.full[stage]);
+                    if constexpr (Cfg<BT, UNPACK>::W8) {
+#pragma unroll
+                        for (int h = 0; h < BK / XBOX; ++h)
+                            ptx::tma_load_2d(sm.wpk[stage] + h * BM * XBOX, &tm_w, kb * BK + h * XBOX, n_tile * BM,
+                                             &sm.full[stage]);
+                    } else {
+                        ptx::tma_load_2d(sm.wpk[stage], &tm_w, kb * (BK / 2), n_tile * BM, &sm.full[stage]);
+                    }
 #pragma unroll
                     for (int h = 0; h < BK / XBOX; ++h)
                         ptx::tma_load_2d(sm.act[stage] + h * BT * XBOX, &tm_x, kb * BK + h * XBOX, m_tile * BT,
@@ -329,32 +356,51 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 ptx::tc_fence_after();
                 const uint8_t *row = sm.wpk[stage] + r * (BK / 2);
                 const int sx_ = r & 7;
+                if constexpr (UNPACK == UNPACK_NONE) {
+                    // W8A8: row r of box `half` holds k in [128 half, +128)
+                    // of the stage, 16-byte chunk c at chunk c ^ (r & 7)
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t out[32];
+                    for (int half = 0; half < 2; ++half) {
+                        const uint8_t *brow = sm.wpk[stage] + half * BM * XBOX + r * XBOX;
+                        uint32_t out[32];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * ((4 * half + c) ^ sx_));
-                        const uint32_t p[4] = {v.x, v.y, v.z, v.w};
+                        for (int c = 0; c < 8; ++c) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(brow + 16 * (c ^ sx_));
+                            out[4 * c] = v.x;
+                            out[4 * c + 1] = v.y;
+                            out[4 * c + 2] = v.z;
+                            out[4 * c + 3] = v.w;
+                        }
+                        ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)(a_col<BT>(slot) + 32 * half), out);
+                    }
+                } else {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint32_t lo, hi;  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
-                            if constexpr (UNPACK == UNPACK_SEXT) {
-                                unpack_s4x8(p[j], lo, hi);
-                            } else {
-                                lo = (p[j] << 4) & 0xF0F0F0F0u;
-                                hi = p[j] & 0xF0F0F0F0u;
-                            }
-                            if constexpr (UNPACK == UNPACK_X16_PERM) {
-                                out[8 * c + 2 * j] = lo;
-                                out[8 * c + 2 * j + 1] = hi;
-                            } else {
-                                out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
-                                out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t out[32];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * ((4 * half + c) ^ sx_));
+                            const uint32_t p[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                uint32_t lo, hi;  // lo = k0,k2,k4,k6; hi = k1,k3,k5,k7
+                                if constexpr (UNPACK == UNPACK_SEXT) {
+                                    unpack_s4x8(p[j], lo, hi);
+                                } else {
+                                    lo = (p[j] << 4) & 0xF0F0F0F0u;
+                                    hi = p[j] & 0xF0F0F0F0u;
+                                }
+                                if constexpr (UNPACK == UNPACK_X16_PERM) {
+                                    out[8 * c + 2 * j] = lo;
+                                    out[8 * c + 2 * j + 1] = hi;
+                                } else {
+                                    out[8 * c + 2 * j] = __byte_perm(lo, hi, 0x5140);      // k0 k1 k2 k3
+                                    out[8 * c + 2 * j + 1] = __byte_perm(lo, hi, 0x7362);  // k4 k5 k6 k7
+                                }
                             }
                         }
+                        ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)(a_col<BT>(slot) + 32 * half), out);
                     }
-                    ptx::tmem_st_32x32b_x32(tmem + lane_base + (uint32_t)(a_col<BT>(slot) + 32 * half), out);
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
@@ -410,7 +456,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 ptx::tmem_wait_ld();
                 const int mrem = M - (m_base + c0);
                 if (mrem <= 0) break;
-                constexpr int SH = UNPACK == UNPACK_SEXT ? 0 : 4;
+                constexpr int SH = Cfg<BT, UNPACK>::SHIFT;
                 const int m0 = m_base + c0;
                 const float *tsx = sm.tsx + c0, *rsx = sm.rsx + c0;
 #define W4A8_EPI(F, B, R) epi_chunk_any<F, B, R, SH>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx)
@@ -482,8 +528,8 @@ inline bool make_map_u8(CUtensorMap *map, const void *base, uint64_t inner, uint
     return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, rows, stride, box_inner, box_rows, swz);
 }
 
-template <int BT>
-inline size_t smem_bytes() { return sizeof(Smem<BT>) + 1024; }
+template <int BT, int UNPACK>
+inline size_t smem_bytes() { return sizeof(Smem<BT, UNPACK>) + 1024; }
 
 template <int BT, int UNPACK>
 inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
@@ -493,12 +539,13 @@ inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(k_gemm_tc<BT, UNPACK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)smem_bytes<BT>());
+                                        (int)smem_bytes<BT, UNPACK>());
     });
     if (attr_err != cudaSuccess) return W4A8_ERR_CUDA;
     CUtensorMap tm_w, tm_x;
-    if (!make_map_u8(&tm_w, Wp, (uint64_t)ldp, (uint64_t)N, (uint64_t)ldp, BK / 2, BM,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+    // W8A8: Wp is the INT8 weight rows, ldp their stride in bytes
+    const uint32_t w_box = Cfg<BT, UNPACK>::W8 ? XBOX : BK / 2;
+    if (!make_map_u8(&tm_w, Wp, (uint64_t)ldp, (uint64_t)N, (uint64_t)ldp, w_box, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_u8(&tm_x, Xq, (uint64_t)ldq, (uint64_t)M, (uint64_t)ldq, XBOX, BT, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     const long long tiles = (long long)((M + BT - 1) / BT) * ((N + BM - 1) / BM);
@@ -506,7 +553,7 @@ inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(NUM_THREADS);
-    cfg.dynamicSmemBytes = smem_bytes<BT>();
+    cfg.dynamicSmemBytes = smem_bytes<BT, UNPACK>();
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -570,6 +617,16 @@ inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const
                                                   sm_count, stream);
     return tc::launch_bt<tc::UNPACK_X16>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
                                          stream);
+}
+
+// W8A8 product on the tensor cores: Wq [N][ldw8] INT8 codes (ldw8 a multiple
+// of 16, bytes k >= K zero), activations in natural k order.
+inline w4a8_status launch_gemm_tc8(const int8_t *Xq, int M, int K, int ldq, const float *sx, const int8_t *Wq,
+                                   int ldw8, const float *sw, int N, const float *bias, unsigned flags, void *Y,
+                                   int ldy, int sm_count, cudaStream_t stream) {
+    const int bt = tc::pick_token_tile(M, N, sm_count);
+    return tc::launch_bt<tc::UNPACK_NONE>(bt, Xq, M, K, ldq, sx, reinterpret_cast<const uint8_t *>(Wq), ldw8, sw, N,
+                                          bias, flags, Y, ldy, sm_count, stream);
 }
 
 }  // namespace w4a8

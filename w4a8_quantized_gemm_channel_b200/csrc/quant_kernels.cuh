@@ -70,9 +70,12 @@ k_col_absmax(const float *__restrict__ W, int K, int N, int ldw, int rows_per_sp
     }
 }
 
+// sw = QMAX / abs-max (1 for an all-zero column): QMAX = 7 for the INT4
+// codes, 127 for the INT8 codes of the W8A8 path.
+template <int QMAX = 7>
 __device__ __forceinline__ float weight_scale_from_amax(unsigned bits) {
     float a = __uint_as_float(bits);
-    return a == 0.0f ? 1.0f : __fdiv_rn(7.0f, a);
+    return a == 0.0f ? 1.0f : __fdiv_rn((float)QMAX, a);
 }
 
 // ---------------------------------------------------------------------------
@@ -144,12 +147,81 @@ k_quant_pack(const float *__restrict__ W, int K, int N, int ldw,
     }
 }
 
+// ---------------------------------------------------------------------------
+// W8A8 weight pass 2 (the INT8 path the guide's INT4 steps extend): codes
+// q = clamp(rne(W[k][n] * sw[n]), -127, 127) with sw = 127 / abs-max, one
+// byte each, rows Wq[n][0, ldw8) with zero pad. A tile is 32 k x (32 * VEC)
+// channels: warp w reads the 4 consecutive rows k0 + 4w .. k0 + 4w + 3
+// (row-coalesced), so each thread holds 4 consecutive codes of each of its
+// channels as one 32-bit word (code k0 + 4w + i in byte i). The words meet
+// in shared memory as [warp][channel] rows; each channel's 8 words (32 k)
+// leave as two 16-byte stores. grid = (ceil(N / (32 * VEC)), ceil(ldw8 / 32)),
+// block = 256.
+// ---------------------------------------------------------------------------
+template <int VEC>
+__global__ void __launch_bounds__(256)
+k_quant8(const float *__restrict__ W, int K, int N, int ldw, const unsigned *__restrict__ amax_bits,
+         int8_t *__restrict__ Wq, int ldw8) {
+    constexpr int COLS = 32 * VEC;
+    __shared__ __align__(16) uint32_t pk[8][COLS];  // [warp][channel]: 4 codes of 4 consecutive k
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nb = blockIdx.x * COLS;
+    const int n = nb + lane * VEC;
+    const int k0 = blockIdx.y * 32 + 4 * warp;
+    float s[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c)
+        s[c] = (n + c < N) ? weight_scale_from_amax<127>(__ldg(amax_bits + n + c)) : 1.0f;
+    float v[4][VEC];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int k = k0 + i;
+        if (k < K && n < N) {
+            if constexpr (VEC == 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4 *>(W + (size_t)k * ldw + n));
+                v[i][0] = f.x; v[i][1] = f.y; v[i][2] = f.z; v[i][3] = f.w;
+            } else {
+                v[i][0] = __ldg(W + (size_t)k * ldw + n);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) v[i][c] = 0.0f;
+        }
+    }
+    uint32_t word[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) {
+        word[c] = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int q = clampi(__float2int_rn(__fmul_rn(v[i][c], s[c])), -127, 127);
+            word[c] |= ((uint32_t)q & 0xFFu) << (8 * i);
+        }
+    }
+    if constexpr (VEC == 4)
+        *reinterpret_cast<uint4 *>(&pk[warp][lane * 4]) = make_uint4(word[0], word[1], word[2], word[3]);
+    else
+        pk[warp][lane] = word[0];
+    __syncthreads();
+    // thread (h, r): channel nb + r, bytes [32 * blockIdx.y + 16h, +16) = the
+    // words of warps 4h .. 4h + 3
+    for (int tt = threadIdx.x; tt < 2 * COLS; tt += 256) {
+        const int r = tt % COLS, h = tt / COLS;
+        const int nn = nb + r;
+        const int byte0 = blockIdx.y * 32 + 16 * h;  // a multiple of 16, as is ldw8
+        if (nn < N && byte0 < ldw8)
+            *reinterpret_cast<uint4 *>(Wq + (size_t)nn * ldw8 + byte0) =
+                make_uint4(pk[4 * h][r], pk[4 * h + 1][r], pk[4 * h + 2][r], pk[4 * h + 3][r]);
+    }
+}
+
 // Weight pass 3: turn the abs-max bits into the scale, in place.
+template <int QMAX = 7>
 __global__ void k_weight_scale_finalize(float *__restrict__ sw, int N) {
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (n < N) {
         unsigned bits = reinterpret_cast<unsigned *>(sw)[n];
-        sw[n] = weight_scale_from_amax(bits);
+        sw[n] = weight_scale_from_amax<QMAX>(bits);
     }
 }
 

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "quant_kernels.cuh"
 #include "linear_simt.cuh"
+#include "linear_w8.cuh"
 #include "decode_bulk.cuh"
 #include "gemm_tc.cuh"
 
@@ -328,6 +329,58 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     return W4A8_OK;
 }
 
+// ------------------------------------------------------------------ W8A8 ---
+// The INT8 path the INT4 steps extend: one INT8 weight code per byte, rows
+// of ldw8 >= K bytes (a multiple of 16), the same argument rules otherwise.
+w4a8_status check_common8(int M, int K, int N, const int8_t *Wq, int ldw8, const float *sw,
+                          const float *bias, unsigned flags, const void *Y, int ldy) {
+    if (K < 1 || K > W8A8_MAX_K || N < 1 || M < 0) return W4A8_ERR_INVALID_ARG;
+    if (!Wq || !aligned16(Wq) || ldw8 < K || ldw8 % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    // the remaining rules are the INT4 layer's (its row check passes for ldw8)
+    return check_common(M, K, N, reinterpret_cast<const uint8_t *>(Wq), ldw8, sw, bias, flags, Y, ldy);
+}
+
+// The W8A8 product on INT8 activations (natural k order).
+w4a8_status run_product8(const int8_t *Xq, int M, int K, int ldq, const float *sx, const int8_t *Wq, int ldw8,
+                         const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                         cudaStream_t stream, bool after_act_pass = false) {
+    const DeviceInfo &dev = device_info();
+    if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
+    const unsigned path = choose_path(M, K, N, flags);
+    cudaError_t e = cudaSuccess;
+    const char *kernel = "";
+    if (path == W4A8_PATH_GENERIC) {
+        kernel = "k_linear8_generic";
+        dim3 grid((N + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
+        e = launch_pdl(k_linear8_generic, grid, dim3(128), 0, stream, Xq, M, K, ldq, sx, Wq, ldw8, sw, N, bias,
+                       flags, Y, ldy);
+    } else if (path == W4A8_PATH_DECODE) {
+        kernel = "k_linear8_decode";
+        const int tok = M <= 8 ? 8 : 16;
+        const int tiles = (M + tok - 1) / tok;
+        if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
+        dim3 grid((N + 15) / 16, tiles);
+        const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
+        auto kern = tok == 8 ? (early ? k_linear8_decode<1, true> : k_linear8_decode<1, false>)
+                             : (early ? k_linear8_decode<2, true> : k_linear8_decode<2, false>);
+        e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream, Xq, M, K, ldq, sx, Wq, ldw8, sw, N, bias, flags,
+                       Y, ldy);
+    } else if (path == W4A8_PATH_TC) {
+        kernel = "k_gemm_tc";
+        if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
+        w4a8_status st = launch_gemm_tc8(Xq, M, K, ldq, sx, Wq, ldw8, sw, N, bias, flags, Y, ldy, dev.sm_count,
+                                         stream);
+        if (st != W4A8_OK) return st;
+    } else {
+        return W4A8_ERR_INVALID_ARG;
+    }
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    t_last_path = path;
+    t_last_launches = 1;
+    t_last_kernel = kernel;
+    return W4A8_OK;
+}
+
 // One launch of the grouped decode kernel over probs[0..count) (count <= 64,
 // every M >= 1).
 template <bool EARLY, int R>
@@ -481,7 +534,44 @@ w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp,
     else
         k_quant_pack<1><<<dim3(col_blocks, kblocks), 256, 0, s>>>(W, K, N, ldw, amax, Wp, ldp);
     if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
-    k_weight_scale_finalize<<<(N + 255) / 256, 256, 0, s>>>(sw, N);
+    k_weight_scale_finalize<7><<<(N + 255) / 256, 256, 0, s>>>(sw, N);
+    return from_cuda(cudaGetLastError());
+}
+
+int w8a8_ld(int K) { return K < 1 ? -1 : round_up(K, 16); }
+
+w4a8_status w8_quantize(const float *W, int K, int N, int ldw, int8_t *Wq, int ldw8, float *sw, void *stream) {
+    if (!W || !Wq || !sw || K < 1 || K > W8A8_MAX_K || N < 1 || ldw < N) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(Wq) || ldw8 < K || ldw8 % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (!aligned4(W) || !aligned4(sw)) return W4A8_ERR_INVALID_ARG;
+    const DeviceInfo &dev = device_info();
+    if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned *amax = reinterpret_cast<unsigned *>(sw);
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * (size_t)N, s);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    const bool v4 = (N % 4 == 0) && (ldw % 4 == 0) && aligned16(W);
+    const int cols = v4 ? 128 : 32;
+    const int col_blocks = (N + cols - 1) / cols;
+    int splits = (6 * dev.sm_count + col_blocks - 1) / col_blocks;
+    splits = splits < 1 ? 1 : splits;
+    int rows = (K + splits - 1) / splits;
+    rows = round_up(rows < 64 ? 64 : rows, 32);
+    splits = (K + rows - 1) / rows;
+    if (splits > 65535) return W4A8_ERR_UNSUPPORTED;
+    if (v4)
+        k_col_absmax<4><<<dim3(col_blocks, splits), 256, 0, s>>>(W, K, N, ldw, rows, amax);
+    else
+        k_col_absmax<1><<<dim3(col_blocks, splits), 256, 0, s>>>(W, K, N, ldw, rows, amax);
+    if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
+    const int kblocks = (ldw8 + 31) / 32;
+    if (kblocks > 65535) return W4A8_ERR_UNSUPPORTED;
+    if (v4)
+        k_quant8<4><<<dim3(col_blocks, kblocks), 256, 0, s>>>(W, K, N, ldw, amax, Wq, ldw8);
+    else
+        k_quant8<1><<<dim3(col_blocks, kblocks), 256, 0, s>>>(W, K, N, ldw, amax, Wq, ldw8);
+    if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
+    k_weight_scale_finalize<127><<<(N + 255) / 256, 256, 0, s>>>(sw, N);
     return from_cuda(cudaGetLastError());
 }
 
@@ -583,6 +673,38 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
     const Workspace ws = carve_workspace(scratch, M, K);
     return linear_from_f32(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, ws,
                            static_cast<cudaStream_t>(stream));
+}
+
+w4a8_status w8a8_linear(const float *X, int M, int K, int ldx, const int8_t *Wq, int ldw8,
+                        const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                        void *workspace, size_t workspace_bytes, void *stream) {
+    w4a8_status st = check_common8(M, K, N, Wq, ldw8, sw, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    if (workspace_bytes < w4a8_workspace_size(M, K)) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    const Workspace ws = carve_workspace(workspace, M, K);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
+    if (st != W4A8_OK) return st;
+    st = run_product8(ws.xq, M, K, ws.ldq, ws.sx, Wq, ldw8, sw, N, bias, flags, Y, ldy, s, true);
+    if (st == W4A8_OK) t_last_launches = 2;
+    return st;
+}
+
+w4a8_status w8a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                          const int8_t *Wq, int ldw8, const float *sw, int N, const float *bias,
+                          unsigned flags, void *Y, int ldy, void *stream) {
+    w4a8_status st = check_common8(M, K, N, Wq, ldw8, sw, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldq < K || ldq % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
+    return run_product8(Xq, M, K, ldq, sx, Wq, ldw8, sw, N, bias, flags, Y, ldy,
+                        static_cast<cudaStream_t>(stream));
 }
 
 unsigned w4a8_last_path(void) { return t_last_path; }

@@ -47,6 +47,10 @@ SIGNATURES = {
     "w4a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
     "w4a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
+    "w8a8_ld": (_I, [_I]),
+    "w8_quantize": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
+    "w8a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
+    "w8a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_last_path": (_U, []),
     "w4a8_last_launch_count": (_U, []),
     "w4a8_last_kernel": (ctypes.c_char_p, []),
@@ -232,6 +236,66 @@ def w4a8_linear_noalloc(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
                                    flags_for(relu, out, path, static_weights), _ptr(y), ldy,
                                    _stream(stream)),
            "w4a8_linear_noalloc")
+    return y
+
+
+# ------------------------------------------------------------------ W8A8 ---
+# The INT8 path the INT4 scheme extends: one INT8 weight code per byte
+# (scale 127 / abs-max), the same activation step and epilogue.
+
+def w8a8_ld(k: int) -> int:
+    return lib.w8a8_ld(k)
+
+
+def w8_quantize(w: torch.Tensor, wq: torch.Tensor | None = None,
+                sw: torch.Tensor | None = None, stream=None):
+    """W[K][N] float32 (CUDA) -> (Wq[N][ldw8] int8, sw[N] float32)."""
+    ldw = _rowmajor(w, "W")
+    k, n = w.shape
+    if wq is None:
+        wq = torch.empty((n, w8a8_ld(k)), dtype=torch.int8, device=w.device)
+    if sw is None:
+        sw = torch.empty(n, dtype=torch.float32, device=w.device)
+    ldw8 = _rowmajor(wq, "Wq")
+    _check(lib.w8_quantize(_ptr(w), k, n, ldw, _ptr(wq), ldw8, _ptr(sw), _stream(stream)), "w8_quantize")
+    return wq, sw
+
+
+def w8a8_linear(x: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
+                path: str = "auto", y: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None,
+                static_weights: bool = False) -> torch.Tensor:
+    """Y[M][N] = dequant(quant8(X) @ Wq^T) (+bias, ReLU) for X[M][K] float32."""
+    ldx = _rowmajor(x, "X")
+    ldw8 = _rowmajor(wq, "Wq")
+    m, k = x.shape
+    n = wq.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, x.device)
+    need = workspace_size(m, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(lib.w8a8_linear(_ptr(x), m, k, ldx, _ptr(wq), ldw8, _ptr(sw), n, _ptr(bias),
+                           flags_for(relu, out, path, static_weights), _ptr(y), ldy, _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream)),
+           "w8a8_linear")
+    return y
+
+
+def w8a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wq: torch.Tensor,
+                  sw: torch.Tensor, bias: torch.Tensor | None = None, relu: bool = False,
+                  out: str = "f32", path: str = "auto", y: torch.Tensor | None = None,
+                  stream=None, static_weights: bool = False) -> torch.Tensor:
+    """Y from INT8 activations Xq[M][ldq] (first k bytes of each row) and sx[M]."""
+    ldq = _rowmajor(xq, "Xq")
+    ldw8 = _rowmajor(wq, "Wq")
+    m = xq.shape[0]
+    n = wq.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, xq.device)
+    _check(lib.w8a8_linear_q(_ptr(xq), m, k, ldq, _ptr(sx), _ptr(wq), ldw8, _ptr(sw), n,
+                             _ptr(bias), flags_for(relu, out, path, static_weights), _ptr(y), ldy,
+                             _stream(stream)),
+           "w8a8_linear_q")
     return y
 
 
