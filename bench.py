@@ -44,6 +44,8 @@ DECODE_TRAFFIC_NOTE = {
     "k_decode_ring": "profiles/k_decode_ring_m1_k4096_n4096.md (M=1)",
     "k_linear_decode": "profiles/launches_decode_bench_k4096_n4096.md (mean of M=4 and M=16)",
 }
+# The same for k_linear8_decode (W8A8 decode), mean over M = 1, 4, 16 (profiles/k_linear8_decode_k4096_n4096.md).
+W8_DECODE_TRAFFIC_PER_LAUNCH = 16834091
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
@@ -123,13 +125,14 @@ class DecodeWorkload:
     outlier channels x20."""
     name = "decode"
 
-    def __init__(self, torch, native, synth, device, l2_bytes):
+    def __init__(self, torch, native, synth, device, l2_bytes, w8=False):
         self.torch, self.nat = torch, native
+        self.w8 = w8  # the W8A8 path: INT8 weight rows instead of packed INT4
         self.K, self.N, self.MS = synth.DECODE_K, synth.DECODE_N, synth.DECODE_MS
         w = synth.decode_case(1).w
         self.w_host = w
         wd = torch.from_numpy(w).to(device)
-        wp, sw = native.w4_quantize_pack(wd)
+        wp, sw = native.w8_quantize(wd) if w8 else native.w4_quantize_pack(wd)
         self.wd = wd
         per_weight = wp.numel() + 4 * sw.numel()
         # enough distinct copies (>= 3x L2) that each launch's weights were
@@ -146,8 +149,14 @@ class DecodeWorkload:
         self.slot = 0
         self.pool_bytes = self.pool * per_weight
 
+    def weight_ld(self):
+        return self.nat.w8a8_ld(self.K) if self.w8 else self.nat.packed_ld(self.K)
+
+    def linear_q(self, *a, **kw):
+        return (self.nat.w8a8_linear_q if self.w8 else self.nat.w4a8_linear_q)(*a, **kw)
+
     def bytes_per_step(self):
-        ldp = self.nat.packed_ld(self.K)
+        ldp = self.weight_ld()
         return sum(self.N * ldp + 4 * self.N + 4 * m * self.K + 4 * m * self.N for m in self.MS)
 
     def ops_per_step(self):
@@ -165,8 +174,9 @@ class DecodeWorkload:
     def call(self, m, s, x=None):
         # weights were quantized before timing and the stream has synchronized
         # since: the serving-style call promises they are settled
-        self.nat.w4a8_linear(self.x[m] if x is None else x, self.wp[s], self.sw[s], y=self.y[m],
-                             workspace=self.ws[m], static_weights=True)
+        lin = self.nat.w8a8_linear if self.w8 else self.nat.w4a8_linear
+        lin(self.x[m] if x is None else x, self.wp[s], self.sw[s], y=self.y[m], workspace=self.ws[m],
+            static_weights=True)
 
     def step(self):
         for m in self.MS:
@@ -175,13 +185,14 @@ class DecodeWorkload:
             self.call(m, s)
 
     def config(self):
-        return {"workload": f"decode single linear K={self.K} N={self.N} M in {list(self.MS)}",
+        return {"workload": f"decode single linear{' W8A8' if self.w8 else ''} K={self.K} N={self.N} "
+                            f"M in {list(self.MS)}",
                 "K": self.K, "N": self.N, "M": list(self.MS),
                 "l2": f"inputs larger than L2: {self.pool} distinct packed weight buffers "
                       f"({self.pool_bytes / 1e6:.0f} MB) rotate across launches",
-                "weights": "N(0,0.02) quantized+packed once before timing",
+                "weights": "N(0,0.02) quantized" + ("" if self.w8 else "+packed") + " once before timing",
                 "activations": "N(0,1), 8 input channels x20",
-                "call": "w4a8_linear with W4A8_STATIC_WEIGHTS"}
+                "call": ("w8a8_linear" if self.w8 else "w4a8_linear") + " with W4A8_STATIC_WEIGHTS"}
 
 
 class PrefillWorkload:
@@ -190,15 +201,16 @@ class PrefillWorkload:
     w4a8_linear (activation quantization + tensor-core GEMM + epilogue)."""
     name = "prefill"
 
-    def __init__(self, torch, native, synth, device, l2_bytes, relu=False):
+    def __init__(self, torch, native, synth, device, l2_bytes, relu=False, w8=False):
         self.torch, self.nat = torch, native
+        self.w8 = w8
         c = synth.prefill_case()
         self.M, self.K, self.N = c.x.shape[0], c.w.shape[0], c.w.shape[1]
         self.MS = (self.M,)
         self.relu = relu
         wd = torch.from_numpy(c.w).to(device)
         self.wd = wd
-        wp, sw = native.w4_quantize_pack(wd)
+        wp, sw = native.w8_quantize(wd) if w8 else native.w4_quantize_pack(wd)
         per_set = wp.numel() + 4 * self.M * self.K + 4 * self.M * self.N
         self.pool = max(2, -(-3 * l2_bytes // per_set))
         self.wp = [wp.clone() for _ in range(self.pool)]
@@ -214,7 +226,8 @@ class PrefillWorkload:
         self.pool_bytes = self.pool * per_set
 
     def bytes_per_step(self):
-        return self.N * self.nat.packed_ld(self.K) + 4 * self.N + 4 * self.M * self.K + 4 * self.M * self.N
+        ldp = self.nat.w8a8_ld(self.K) if self.w8 else self.nat.packed_ld(self.K)
+        return self.N * ldp + 4 * self.N + 4 * self.M * self.K + 4 * self.M * self.N
 
     def ops_per_step(self):
         return 2 * self.M * self.N * self.K
@@ -225,12 +238,12 @@ class PrefillWorkload:
     def step(self):
         s = self.slot
         self.slot = (self.slot + 1) % self.pool
-        self.nat.w4a8_linear(self.xs[s], self.wp[s], self.sw[s], relu=self.relu, y=self.ys[s],
-                             workspace=self.ws[self.M])
+        lin = self.nat.w8a8_linear if self.w8 else self.nat.w4a8_linear
+        lin(self.xs[s], self.wp[s], self.sw[s], relu=self.relu, y=self.ys[s], workspace=self.ws[self.M])
 
     def config(self):
-        return {"workload": f"prefill single linear M={self.M} K={self.K} N={self.N}"
-                            + (" +ReLU" if self.relu else ""),
+        return {"workload": f"prefill single linear{' W8A8' if self.w8 else ''} M={self.M} K={self.K} "
+                            f"N={self.N}" + (" +ReLU" if self.relu else ""),
                 "M": self.M, "K": self.K, "N": self.N,
                 "l2": f"inputs larger than L2: {self.pool} distinct X/W/Y sets "
                       f"({self.pool_bytes / 1e6:.0f} MB) rotate across launches"}
@@ -302,15 +315,15 @@ def time_kernel_only(torch, nat, wl):
     weight pool, per M; returns {m: (ms_per_launch, algorithmic_bytes,
     kernel_name)}."""
     out = {}
-    ldp = nat.packed_ld(wl.K)
+    ldp = wl.weight_ld()
     for m in wl.MS:
         xq, sx = nat.a8_quantize_rows(wl.x[m])
         reps = wl.pool
 
         def run():
             for i in range(reps):
-                nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], y=wl.y[m], static_weights=True)
-        nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[0], wl.sw[0], y=wl.y[m], static_weights=True)
+                wl.linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], y=wl.y[m], static_weights=True)
+        wl.linear_q(xq, sx, wl.K, wl.wp[0], wl.sw[0], y=wl.y[m], static_weights=True)
         kernel = nat.last_kernel()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
@@ -341,10 +354,11 @@ def time_gemm_only(torch, nat, wl, reps=20):
     activations) over the rotating buffer sets."""
     m = wl.M
     xqs = [nat.a8_quantize_rows(x) for x in wl.xs]
+    lin_q = nat.w8a8_linear_q if wl.w8 else nat.w4a8_linear_q
     def run():
         for i in range(wl.pool):
             xq, sx = xqs[i]
-            nat.w4a8_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
+            lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
@@ -454,8 +468,8 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False):
-    wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu)
+def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False):
+    wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu, w8=w8)
     clocks = ClockSampler(device.index or 0)
     clocks.start()
     time.sleep(0.3)
@@ -469,14 +483,53 @@ def run_prefill(args, torch, native, synth, device, props, dist, world, rank, re
     achieved = wl.ops_per_step() / (g_ms * 1e-3) / 1e12
     line = {"metric": METRIC, "value": round(tops, 2), "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8xs4->s32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "s8xs8->s32" if w8 else "s8xs4->s32",
             "data": "synthetic", "config": wl.config(),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                          "unit": "TOPS", "frac": round(achieved / peak, 4),
                          "peak_source": f"{kind} bf16_tflops x {INT8_OVER_BF16:g} (nominal int8/bf16)",
-                         "traffic": None, "kernel": "k_gemm_tc (w4a8_linear_q, rotating buffers)",
+                         "traffic": None, "kernel": "k_gemm_tc (" + ("w8a8" if w8 else "w4a8")
+                                                    + "_linear_q, rotating buffers)",
                          "us": round(g_ms * 1e3, 2)},
             "gpu_launches": args.steps * wl.launches_per_step(), "clocks": ck}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank):
+    """The decode workload on the W8A8 path: the step (w8a8_linear at M = 1,
+    4, 16, activation pass included) and the product kernel alone per M."""
+    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size, w8=True)
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_steps(torch, wl, args.steps, args.warmup, dist)
+    ck = clocks.stop()
+    ms = max_over_ranks(torch, dist, ms, device)
+    bytes_step = wl.bytes_per_step()
+    value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9
+    kern = time_kernel_only(torch, native, wl)
+    k_ms = sum(v[0] for v in kern.values())
+    k_bytes = sum(v[1] for v in kern.values())
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    achieved = k_bytes / (k_ms * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8xs8->s32",
+            "data": "synthetic", "config": wl.config(),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
+                         "traffic": W8_DECODE_TRAFFIC_PER_LAUNCH,
+                         "traffic_note": "dram bytes read+written per k_linear8_decode launch, mean over M = 1, "
+                                         "4, 16; ncu capture in profiles/k_linear8_decode_k4096_n4096.md",
+                         "kernel": "k_linear8_decode over M in " + str(list(kern)) + " (w8a8_linear_q "
+                                   "back-to-back over rotating weights, static-weights promise)",
+                         "per_m": {str(m): {"kernel": v[2], "us": round(v[0] * 1e3, 3), "bytes": v[1],
+                                            "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
+                                   for m, v in kern.items()}},
+            "gpu_launches": args.steps * 2 * len(wl.MS), "clocks": ck}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -672,10 +725,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU work for the oracle baseline")
-    ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep", "gemma-stack"],
+    ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep", "gemma-stack",
+                                           "decode-w8a8", "prefill-w8a8"],
                     default="decode",
                     help="decode (the headline line), prefill (M=2048 K=4096 N=11008), a per-shape "
-                         "sweep of the other workloads, or the 182-linear Gemma3-1B-shaped stack")
+                         "sweep of the other workloads, the 182-linear Gemma3-1B-shaped stack, or the "
+                         "decode / prefill workloads on the W8A8 path")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -710,9 +765,12 @@ def main():
 
     from w4a8_quantized_gemm_channel_b200 import native, synth
     props = torch.cuda.get_device_properties(device)
-    if args.workload in ("prefill", "prefill-relu"):
+    if args.workload in ("prefill", "prefill-relu", "prefill-w8a8"):
         run_prefill(args, torch, native, synth, device, props, dist, world, rank,
-                    relu=args.workload == "prefill-relu")
+                    relu=args.workload == "prefill-relu", w8=args.workload == "prefill-w8a8")
+        return
+    if args.workload == "decode-w8a8":
+        run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank)
         return
     if args.workload == "sweep":
         run_sweep(torch, native, synth, device, props)

@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -54,9 +55,11 @@ template <> struct Ring<192> { static constexpr int STAGES = 3, A_SLOTS = 2; }; 
 template <> struct Ring<128> { static constexpr int STAGES = 4, A_SLOTS = 4; };  // 4 x 48 KB, 256 + 256 cols
 template <> struct Ring<64> { static constexpr int STAGES = 6, A_SLOTS = 4; };   // 6 x 32 KB, 128 + 256 cols
 // The W8A8 form: weight tiles of one byte per code are twice as large, so
-// fewer stages fit the same shared memory.
+// fewer stages fit the same shared memory. A 192-token tile would keep only
+// 2 stages of 80 KB; measured on B200 that ring was too shallow (1194 TOPS at
+// M = 2048, K = 4096, N = 11008 against 1622 with BT = 128), so W8A8 runs
+// BT = 128 or 64 only.
 template <int BT> struct Ring8;
-template <> struct Ring8<192> { static constexpr int STAGES = 2, A_SLOTS = 2; };  // 2 x 80 KB, 384 + 128 cols
 template <> struct Ring8<128> { static constexpr int STAGES = 3, A_SLOTS = 2; };  // 3 x 64 KB, 256 + 128 cols
 template <> struct Ring8<64> { static constexpr int STAGES = 4, A_SLOTS = 4; };   // 4 x 48 KB, 128 + 256 cols
 // Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
@@ -91,8 +94,9 @@ constexpr int TC_X16_MAX_K = 131072;
 template <int BT, int UNPACK>
 struct Cfg {
     static constexpr bool W8 = UNPACK == UNPACK_NONE;
-    static constexpr int STAGES = W8 ? Ring8<BT>::STAGES : Ring<BT>::STAGES;
-    static constexpr int A_SLOTS = W8 ? Ring8<BT>::A_SLOTS : Ring<BT>::A_SLOTS;
+    using R = std::conditional_t<W8, Ring8<BT>, Ring<BT>>;
+    static constexpr int STAGES = R::STAGES;
+    static constexpr int A_SLOTS = R::A_SLOTS;
     static constexpr int W_TILE_BYTES = W8 ? BM * BK : BM * BK / 2;
     static constexpr int SHIFT = (UNPACK == UNPACK_X16 || UNPACK == UNPACK_X16_PERM) ? 4 : 0;
 };
@@ -576,11 +580,12 @@ namespace tc {
 // Token tile for a call: the one with the smallest estimated time, where a
 // round of tiles over the SMs costs ceil(K / BK) iterations of about
 // 8 x BT / 2 tensor cycles plus ~600 cycles of per-iteration overhead.
-inline int pick_token_tile(int M, int N, int sm_count) {
+inline int pick_token_tile(int M, int N, int sm_count, bool allow192 = true) {
     const int cand[3] = {192, 128, 64};
-    int best = 192;
+    int best = allow192 ? 192 : 128;
     long long best_cost = -1;
     for (int bt : cand) {
+        if (bt == 192 && !allow192) continue;
         const long long tiles = (long long)((M + bt - 1) / bt) * ((N + BM - 1) / BM);
         const long long rounds = (tiles + sm_count - 1) / sm_count;
         const long long cost = rounds * (8LL * bt / 2 + 600);
@@ -624,9 +629,11 @@ inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const
 inline w4a8_status launch_gemm_tc8(const int8_t *Xq, int M, int K, int ldq, const float *sx, const int8_t *Wq,
                                    int ldw8, const float *sw, int N, const float *bias, unsigned flags, void *Y,
                                    int ldy, int sm_count, cudaStream_t stream) {
-    const int bt = tc::pick_token_tile(M, N, sm_count);
-    return tc::launch_bt<tc::UNPACK_NONE>(bt, Xq, M, K, ldq, sx, reinterpret_cast<const uint8_t *>(Wq), ldw8, sw, N,
-                                          bias, flags, Y, ldy, sm_count, stream);
+    const int bt = tc::pick_token_tile(M, N, sm_count, false);
+    const uint8_t *w = reinterpret_cast<const uint8_t *>(Wq);
+    if (bt == 64)
+        return tc::launch<64, tc::UNPACK_NONE>(Xq, M, K, ldq, sx, w, ldw8, sw, N, bias, flags, Y, ldy, sm_count, stream);
+    return tc::launch<128, tc::UNPACK_NONE>(Xq, M, K, ldq, sx, w, ldw8, sw, N, bias, flags, Y, ldy, sm_count, stream);
 }
 
 }  // namespace w4a8
