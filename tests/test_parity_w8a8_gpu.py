@@ -146,3 +146,19 @@ def test_w8a8_prefill_full_size_sampled(nat):
     assert np.array_equal(acc[np.ix_(rows, cols)], oracle.linear8(c.x[rows], q8_s, sw_s, k, out="s32"))
     y = host(nat.w8a8_linear(dev(c.x), wqd, swd, relu=True))
     assert_f32_close(y[np.ix_(rows, cols)], oracle.linear8(c.x[rows], q8_s, sw_s, k, relu=True))
+
+
+@pytest.mark.parametrize("m,k,n", [(1024, 520, 4096), (2048, 777, 11008), (333, 1040, 2000)])
+def test_w8a8_tc_token_tiles_sampled(nat, m, k, n):
+    """Shapes on which the tensor-core GEMM's tile estimate picks each of its
+    W8A8 token tiles (128, 160, and 64 with a ragged last tile): sampled
+    rows x channels, INT32 bit for bit."""
+    x, w, _ = _case(m, k, n, seed=2500 + m)
+    wqd, swd = nat.w8_quantize(dev(w))
+    rng = synth.rng_for(2500, m)
+    rows = np.sort(rng.choice(m, 20, replace=False))
+    rows[-1] = m - 1  # the last row of the last (ragged) token tile
+    cols = np.sort(rng.choice(n, 80, replace=False))
+    q8_s, sw_s = oracle.w8_quantize(w[:, cols])
+    acc = host(nat.w8a8_linear(dev(x), wqd, swd, out="s32", path="tc"))
+    assert np.array_equal(acc[np.ix_(rows, cols)], oracle.linear8(x[rows], q8_s, sw_s, k, out="s32"))

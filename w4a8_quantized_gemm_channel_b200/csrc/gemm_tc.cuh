@@ -60,6 +60,7 @@ template <> struct Ring<64> { static constexpr int STAGES = 6, A_SLOTS = 4; };  
 // M = 2048, K = 4096, N = 11008 against 1622 with BT = 128), so W8A8 runs
 // BT = 128 or 64 only.
 template <int BT> struct Ring8;
+template <> struct Ring8<160> { static constexpr int STAGES = 3, A_SLOTS = 2; };  // 3 x 72 KB, 320 + 128 cols
 template <> struct Ring8<128> { static constexpr int STAGES = 3, A_SLOTS = 2; };  // 3 x 64 KB, 256 + 128 cols
 template <> struct Ring8<64> { static constexpr int STAGES = 4, A_SLOTS = 4; };   // 4 x 48 KB, 128 + 256 cols
 // Unpack warpgroups: pipeline iteration `it` is unpacked by warpgroup
@@ -580,12 +581,12 @@ namespace tc {
 // Token tile for a call: the one with the smallest estimated time, where a
 // round of tiles over the SMs costs ceil(K / BK) iterations of about
 // 8 x BT / 2 tensor cycles plus ~600 cycles of per-iteration overhead.
-inline int pick_token_tile(int M, int N, int sm_count, bool allow192 = true) {
-    const int cand[3] = {192, 128, 64};
-    int best = allow192 ? 192 : 128;
+inline int pick_token_tile(int M, int N, int sm_count, bool w8 = false) {
+    const int cand[4] = {192, 160, 128, 64};
+    int best = w8 ? 160 : 192;
     long long best_cost = -1;
     for (int bt : cand) {
-        if (bt == 192 && !allow192) continue;
+        if (bt == (w8 ? 192 : 160)) continue;  // INT4 forms: 192/128/64; W8A8: 160/128/64
         const long long tiles = (long long)((M + bt - 1) / bt) * ((N + BM - 1) / BM);
         const long long rounds = (tiles + sm_count - 1) / sm_count;
         const long long cost = rounds * (8LL * bt / 2 + 600);
@@ -629,11 +630,14 @@ inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const
 inline w4a8_status launch_gemm_tc8(const int8_t *Xq, int M, int K, int ldq, const float *sx, const int8_t *Wq,
                                    int ldw8, const float *sw, int N, const float *bias, unsigned flags, void *Y,
                                    int ldy, int sm_count, cudaStream_t stream) {
-    const int bt = tc::pick_token_tile(M, N, sm_count, false);
+    const int bt = tc::pick_token_tile(M, N, sm_count, true);
     const uint8_t *w = reinterpret_cast<const uint8_t *>(Wq);
     if (bt == 64)
         return tc::launch<64, tc::UNPACK_NONE>(Xq, M, K, ldq, sx, w, ldw8, sw, N, bias, flags, Y, ldy, sm_count, stream);
-    return tc::launch<128, tc::UNPACK_NONE>(Xq, M, K, ldq, sx, w, ldw8, sw, N, bias, flags, Y, ldy, sm_count, stream);
+    if (bt == 128)
+        return tc::launch<128, tc::UNPACK_NONE>(Xq, M, K, ldq, sx, w, ldw8, sw, N, bias, flags, Y, ldy, sm_count,
+                                                stream);
+    return tc::launch<160, tc::UNPACK_NONE>(Xq, M, K, ldq, sx, w, ldw8, sw, N, bias, flags, Y, ldy, sm_count, stream);
 }
 
 }  // namespace w4a8
