@@ -267,7 +267,8 @@ W4A8_API w4a8_status w8a8_linear_q(const int8_t *Xq, int M, int K, int ldq, cons
                           const float *bias, unsigned flags, void *Y, int ldy, void *stream);
 
 /* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
- * last successful w4a8_linear / w4a8_linear_q call enqueued; 0 if none. */
+ * last successful w4a8_linear / w4a8_linear_q / w8a8_linear / w8a8_linear_q
+ * call enqueued (grouped calls: _DECODE); 0 if none. */
 W4A8_API unsigned w4a8_last_path(void);
 
 /* How many kernels the calling thread's last successful w4a8_linear /
@@ -276,9 +277,11 @@ W4A8_API unsigned w4a8_last_path(void);
 W4A8_API unsigned w4a8_last_launch_count(void);
 
 /* Name of the product kernel that the calling thread's last successful
- * w4a8_linear / w4a8_linear_q / w4a8_linear_noalloc / w4a8_linear_grouped
+ * w4a8_linear / w4a8_linear_q / w4a8_linear_noalloc / w4a8_linear_grouped /
+ * w8a8_linear / w8a8_linear_q
  * call enqueued ("k_decode_ring", "k_linear_decode", "k_gemm_tc",
- * "k_linear_generic" or "k_decode_grouped"), not counting the activation
+ * "k_linear_generic", "k_decode_grouped", or for the W8A8 calls
+ * "k_linear8_decode", "k_linear8_generic", "k_gemm_tc"), not counting the activation
  * pass; "" if none, or if that call had nothing to do. A static string that
  * the caller must not free. */
 W4A8_API const char *w4a8_last_kernel(void);

@@ -139,9 +139,9 @@ bool raise_smem_limit(const void *kern, int bytes) {
     return true;
 }
 
-// The persistent decode kernel (one block per SM, a TMA ring of weight
-// stages) serves M <= 8 when its ring and the activation rows fit the
-// shared-memory budget.
+// The persistent decode kernel (a TMA ring of weight stages) serves M <= 8
+// when its ring and the activation rows fit the shared-memory budget, except
+// where registers_beat_ring hands a short layer to k_linear_decode.
 struct RingPlan {
     bool ok = false;
     int grid = 0, ring_n = 0;
