@@ -67,6 +67,8 @@ def _load():
                 "oracle_quantize_weight": [ctypes.c_float, ctypes.c_float],
                 "oracle_w8_quantize": [P, I, I, I, P, I, P],
                 "oracle_gemm8_s32": [P, I, I, I, P, I, I, P, I],
+                "oracle_w4z_quantize_pack": [P, I, I, I, P, I, P, P],
+                "oracle_gemm_z_s32": [P, I, I, I, P, I, I, P, P, I],
             }.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
@@ -264,6 +266,50 @@ def linear8_q(xq: np.ndarray, sx: np.ndarray, q8: np.ndarray, sw: np.ndarray, k:
     if out == "s32":
         return acc
     y = dequant(acc, sx, sw, bias, relu)
+    return to_bf16_bits(y) if out == "bf16" else y
+
+
+# ------------------------------------------------ asymmetric INT4 (zero point) ---
+# Uniform asymmetric quantization of the weights per output channel ("INT4"
+# concept page, section 4.1; "4-bit Integer Quantization for LLMs" page,
+# section "Weight quantization"): multiplier sa = 15 / (max - min), integer
+# zero point zp = -rne(min * sa), codes q = clamp(rne(w * sa) + zp, 0, 15)
+# packed as unsigned nibbles; activations as in step 3.
+
+def w4z_quantize_pack(w: np.ndarray, ldp: int | None = None):
+    """W[K][N] float32 -> (Wp[N][ldp] uint8, sa[N] float32, zp[N] int32)."""
+    w = _f32(w)
+    k, n = w.shape
+    ldp = packed_ld(k) if ldp is None else ldp
+    wp = np.empty((n, ldp), np.uint8)
+    sa = np.empty(n, np.float32)
+    zp = np.empty(n, np.int32)
+    _check(_load().oracle_w4z_quantize_pack(_ptr(w), k, n, n, _ptr(wp), ldp, _ptr(sa), _ptr(zp)),
+           "w4z_quantize_pack")
+    return wp, sa, zp
+
+
+def gemm_z_s32(xq: np.ndarray, k: int, wp: np.ndarray, zp: np.ndarray) -> np.ndarray:
+    """acc[M][N] = sum_k xq[m][k] * (q[n][k] - zp[n]) (exact, must fit INT32)."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    wp = np.ascontiguousarray(wp, dtype=np.uint8)
+    zp = np.ascontiguousarray(zp, dtype=np.int32)
+    m, ldq = xq.shape
+    n, ldp = wp.shape
+    acc = np.empty((m, n), np.int32)
+    _check(_load().oracle_gemm_z_s32(_ptr(xq), m, k, ldq, _ptr(wp), n, ldp, _ptr(zp), _ptr(acc), n),
+           "gemm_z_s32")
+    return acc
+
+
+def linear_z(x: np.ndarray, wp: np.ndarray, sa: np.ndarray, zp: np.ndarray, k: int,
+             bias: np.ndarray | None = None, relu: bool = False, out: str = "f32"):
+    """One Dense layer with zero-point INT4 weights on float32 input."""
+    xq, sx = a8_quantize_rows(x)
+    acc = gemm_z_s32(xq, k, wp, zp)
+    if out == "s32":
+        return acc
+    y = dequant(acc, sx, sa, bias, relu)
     return to_bf16_bits(y) if out == "bf16" else y
 
 

@@ -28,6 +28,19 @@
  * step: sw = 127 / max|W[:,n]| (1 for a zero column), q = clamp(rne(w * sw),
  * -127, 127), one byte per code, rows of ldw8 >= K bytes with zero pad.
  *
+ * Asymmetric INT4 with a zero point (the uniform quantization of the "INT4"
+ * concept page, section 4.1, asymmetric form; the formulas of the "4-bit
+ * Integer Quantization for LLMs" page, section "Weight quantization"), per
+ * output channel, with the activations as in step 3. The pages give
+ * scale = (max - min) / (2^4 - 1), q = round(w / scale) + zero_point in
+ * [0, 15] and w ~ (q - zero_point) * scale. Read here as: the multiplier
+ * sa = 15 / (max - min) (1 when max == min) in place of the division, like
+ * the symmetric scale; the integer zero point zp = -rne(min * sa), so that
+ * the minimum maps to code 0; q = clamp(rne(w * sa) + zp, 0, 15) (the clamp
+ * binds only when a tie lifts the maximum to 16); codes packed unsigned, two
+ * per byte along K, even k in the low nibble; the product
+ * acc = sum_k xq * (q - zp) and y = float(acc) / (sx * sa).
+ *
  * Precision: the page's model is float32 end to end (its inputs are cast with
  * astype("float32")), and float32 decides every integer code, so each step
  * below runs in float32 with IEEE round-to-nearest. Build flags:
@@ -301,6 +314,68 @@ int oracle_gemm8_s32(const int8_t *Xq, int M, int K, int ldq,
             int64_t s = 0;
             for (int k = 0; k < K; ++k)
                 s += (int64_t)Xq[(size_t)m * ldq + k] * (int64_t)Q8[(size_t)n * ldw8 + k];
+            if (s > INT32_MAX || s < INT32_MIN) return ORACLE_OVERFLOW;
+            acc[(size_t)m * ldacc + n] = (int32_t)s;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Asymmetric INT4 with a zero point, steps 1-2 per output channel:
+ * sa[n] = 15 / (max_k W[k][n] - min_k W[k][n]) (1 when they are equal),
+ * zp[n] = -rne(min_k W[k][n] * sa[n]), q = clamp(rne(w * sa[n]) + zp[n], 0, 15),
+ * packed as unsigned nibbles: byte j of row n = q[2j] | q[2j+1] << 4, every
+ * byte past the nibble of k = K-1 zero.
+ * ------------------------------------------------------------------------- */
+int oracle_w4z_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp, int ldp,
+                             float *sa, int32_t *zp)
+{
+    if (!W || !Wp || !sa || !zp || K < 1 || N < 1 || ldw < N || ldp < (K + 1) / 2) return ORACLE_BAD_ARG;
+    for (int n = 0; n < N; ++n) {
+        float lo = W[n], hi = W[n];
+        for (int k = 1; k < K; ++k) {
+            float w = W[(size_t)k * ldw + n];
+            if (w < lo) lo = w;
+            if (w > hi) hi = w;
+        }
+        float range = hi - lo;
+        sa[n] = (range == 0.0f) ? 1.0f : 15.0f / range;
+        zp[n] = -(int32_t)round_half_even(lo * sa[n]);
+        uint8_t *row = Wp + (size_t)n * ldp;
+        memset(row, 0, (size_t)ldp);
+        for (int k = 0; k < K; ++k) {
+            float t = W[(size_t)k * ldw + n] * sa[n];
+            int q = clamp_int((int)round_half_even(t) + zp[n], 0, 15);
+            if (k % 2 == 0)
+                row[k / 2] |= (uint8_t)q;
+            else
+                row[k / 2] |= (uint8_t)(q << 4);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* The unsigned code of nibble k of packed row n (zero-point layout). */
+static int zp_code(const uint8_t *Wp, int ldp, int n, int k)
+{
+    uint8_t byte = Wp[(size_t)n * ldp + k / 2];
+    return (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+}
+
+/* acc[m][n] = sum_k xq[m][k] * (q[n][k] - zp[n]), exact (int64) and required
+ * to fit INT32. */
+int oracle_gemm_z_s32(const int8_t *Xq, int M, int K, int ldq, const uint8_t *Wp, int N, int ldp,
+                      const int32_t *zp, int32_t *acc, int ldacc)
+{
+    if (M < 0 || K < 1 || N < 1 || ldq < K || ldp < (K + 1) / 2 || ldacc < N) return ORACLE_BAD_ARG;
+    if (M == 0) return ORACLE_OK;
+    if (!Xq || !Wp || !zp || !acc) return ORACLE_BAD_ARG;
+    for (int m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            int64_t s = 0;
+            for (int k = 0; k < K; ++k)
+                s += (int64_t)Xq[(size_t)m * ldq + k] * (int64_t)(zp_code(Wp, ldp, n, k) - zp[n]);
             if (s > INT32_MAX || s < INT32_MIN) return ORACLE_OVERFLOW;
             acc[(size_t)m * ldacc + n] = (int32_t)s;
         }

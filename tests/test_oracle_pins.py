@@ -420,3 +420,113 @@ def test_linear8_error_bound_and_tighter_than_int4():
     wp, sw4 = oracle.w4_quantize_pack(w)
     y4 = oracle.linear(x, wp, sw4, 640)
     assert np.abs(y8 - exact).mean() < 0.5 * np.abs(y4 - exact).mean()
+
+
+# ------------------------------------------------ asymmetric INT4 (zero point) ---
+# "INT4" concept page, section 4.1 (asymmetric uniform quantization) and the
+# "4-bit Integer Quantization for LLMs" page, section "Weight quantization".
+
+def _unpack_unsigned(wp, k):
+    """Nibbles of each packed row as unsigned codes, written independently of the oracle."""
+    lo = (wp & 0x0F).astype(np.int64)
+    hi = (wp >> 4).astype(np.int64)
+    codes = np.empty((wp.shape[0], 2 * wp.shape[1]), np.int64)
+    codes[:, 0::2], codes[:, 1::2] = lo, hi
+    return codes[:, :k]
+
+
+def test_w4z_hand_worked_codes():
+    """Column [-1, 0, 2, 0.5]: range 3 -> sa = 15/3 = 5, zp = -rne(-5) = 5;
+    codes -5+5 = 0, 0+5 = 5, 10+5 = 15, rne(2.5) = 2 (tie to even) + 5 = 7;
+    bytes 0 | 5 << 4 = 80 and 15 | 7 << 4 = 127, pad 0."""
+    w = np.array([[-1.0], [0.0], [2.0], [0.5]], np.float32)
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    assert sa.tolist() == [5.0] and zp.tolist() == [5]
+    assert wp[0, :2].tolist() == [80, 127] and not wp[0, 2:].any()
+
+
+def test_w4z_clamp_binds_on_a_tie_at_the_top():
+    """Column [-0.5, 0.5, 0]: sa = 15, zp = -rne(-7.5) = 8 (tie to even);
+    0.5 * 15 = 7.5 also rounds to 8, and 8 + 8 = 16 must clamp to 15 (not wrap
+    to 0); 0 maps to 8. Bytes 0 | 15 << 4 = 240 and 8."""
+    w = np.array([[-0.5], [0.5], [0.0]], np.float32)
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    assert sa.tolist() == [15.0] and zp.tolist() == [8]
+    assert wp[0, :2].tolist() == [240, 8]
+
+
+def test_w4z_range_ends_and_dequant_error():
+    """Each column's minimum maps to code 0 and its maximum to 15; every code is
+    in [0, 15]; the dequantized weight (q - zp) / sa is within 0.5 / sa of w
+    except where the clamp took a tie at the top from 16 to 15 (then 1 / sa)."""
+    w = _random_w(k=300, n=40, seed=41)
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    q = _unpack_unsigned(wp, 300)
+    assert q.min() >= 0 and q.max() <= 15
+    for n in range(40):
+        assert q[n, int(np.argmin(w[:, n]))] == 0 and q[n, int(np.argmax(w[:, n]))] == 15
+    deq = (q - zp[:, None].astype(np.int64)) / sa.astype(np.float64)[:, None]
+    err = np.abs(w.T.astype(np.float64) - deq)
+    step = 1.0 / sa.astype(np.float64)[:, None]
+    assert (err <= step * (1 + 1e-6)).all()
+    assert (err <= 0.5 * step * (1 + 1e-6)).mean() > 0.99
+
+
+def test_w4z_scale_is_15_over_range_and_power_of_two_invariance():
+    w = _random_w(k=200, n=8, seed=42)
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    rng_ = (w.max(axis=0) - w.min(axis=0)).astype(np.float32)
+    assert np.array_equal(sa, (np.float32(15.0) / rng_).astype(np.float32))
+    for j in (-3, 2):
+        wj, saj, zpj = oracle.w4z_quantize_pack((w * np.float32(2.0 ** j)).astype(np.float32))
+        assert np.array_equal(wj, wp) and np.array_equal(zpj, zp)
+        assert np.array_equal(saj * np.float32(2.0 ** j), sa)
+
+
+def test_w4z_constant_and_positive_columns():
+    """A constant column c has no range: sa = 1, zp = -rne(c), all codes 0,
+    dequantized rne(c). An all-positive column gets a negative zero point and
+    still spans codes 0..15."""
+    w = np.zeros((6, 2), np.float32)
+    w[:, 0] = 3.25
+    w[:, 1] = [100.0, 100.2, 100.4, 100.6, 100.8, 101.0]
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    assert sa[0] == 1.0 and zp[0] == -3 and not (wp[0] & 0x0F).any() and not (wp[0] >> 4).any()
+    q = _unpack_unsigned(wp, 6)
+    assert zp[1] < 0 and q[1, 0] == 0 and q[1, 5] == 15
+
+
+def test_gemm_z_matches_float64_matmul():
+    """sum_k xq * (q - zp) against float64 matmul of independently unpacked
+    codes (exact while |acc| < 2^53)."""
+    rng = synth.rng_for(43, 0)
+    for (m, k, n) in ((1, 1, 1), (3, 7, 5), (24, 777, 40)):
+        w = rng.normal(0.0, 0.02, size=(k, n)).astype(np.float32)
+        wp, sa, zp = oracle.w4z_quantize_pack(w)
+        xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+        acc = oracle.gemm_z_s32(xq, k, wp, zp)
+        q = _unpack_unsigned(wp, k) - zp[:, None].astype(np.int64)
+        assert np.array_equal(acc.astype(np.float64), xq.astype(np.float64) @ q.T.astype(np.float64))
+
+
+def test_linear_z_error_bound_and_tighter_than_symmetric():
+    """|y - X @ W| within the bound with e_w = 1 / sa (the clamp case) and
+    e_x = 0.5 / sx; and since the asymmetric grid spends all 16 levels on each
+    column's range, its mean error on the same data is below the symmetric
+    layer's (which uses 15 of 16 levels over twice the abs-max)."""
+    x, _ = synth.linear_activations(8, 640, seed=44, outlier_count=3, outlier_factor=20.0)
+    w = synth.linear_weights(640, 48, 0.02, seed=44)
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    xq, sx = oracle.a8_quantize_rows(x)
+    y = oracle.linear_z(x, wp, sa, zp, 640)
+    x64, w64 = x.astype(np.float64), w.astype(np.float64)
+    exact = x64 @ w64
+    ew = 1.0 / sa.astype(np.float64)
+    ex = 0.5 / sx.astype(np.float64)
+    bound = (np.abs(x64).sum(1)[:, None] * ew[None, :] + ex[:, None] * np.abs(w64).sum(0)[None, :]
+             + 640 * ex[:, None] * ew[None, :])
+    slack = 1e-5 * (np.abs(x64) @ np.abs(w64)) + 1e-6
+    assert (np.abs(y - exact) <= bound + slack).all()
+    wps, sws = oracle.w4_quantize_pack(w)
+    ys = oracle.linear(x, wps, sws, 640)
+    assert np.abs(y - exact).mean() < np.abs(ys - exact).mean()
