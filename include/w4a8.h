@@ -266,6 +266,55 @@ W4A8_API w4a8_status w8a8_linear_q(const int8_t *Xq, int M, int K, int ldq, cons
                           const int8_t *Wq, int ldw8, const float *sw, int N,
                           const float *bias, unsigned flags, void *Y, int ldy, void *stream);
 
+/*
+ * Zero-point INT4 - asymmetric per-output-channel weights (the uniform
+ * asymmetric quantization of the "INT4" concept page, section 4.1, and the
+ * formulas of the "4-bit Integer Quantization for LLMs" page, section "Weight
+ * quantization"), with the activation step, product and epilogue of the W4A8
+ * layer:
+ *   sa[n] = 15 / (max_k W[k][n] - min_k W[k][n])  (1 when they are equal),
+ *   zp[n] = -rne(min_k W[k][n] * sa[n]),  q = clamp(rne(w * sa[n]) + zp[n], 0, 15),
+ *   acc = sum_k xq[m][k] * (q - zp[n]),  y = float(acc) / (sx[m] * sa[n]).
+ * Storage: Wp as for w4_quantize_pack ([N][ldp] bytes, two nibbles per byte,
+ * even k low) holding each code as the signed nibble q - 8 (q XOR 8), pad
+ * nibbles 0; the W4A8 kernels multiply those and an epilogue adds
+ * -(zp - 8) * sum_k xq[m][k]. Results are defined while acc fits INT32.
+ */
+
+/*
+ * w4z_quantize_pack - steps 1-2 of the zero-point form.
+ *   W  [K][ldw] float32 (the Keras kernel layout), ldw >= N, finite.
+ *   Wp [N][ldp] bytes out (ldp >= ceil(K/2), a multiple of 16, 16-byte aligned).
+ *   sa [N] float32 out, zp [N] int32 out (both used as scratch while it runs).
+ * Requires 1 <= K <= W4A8_MAX_K, N >= 1.
+ */
+W4A8_API w4a8_status w4z_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp, int ldp,
+                              float *sa, int32_t *zp, void *stream);
+
+/* Workspace bytes of w4z_linear / w4z_linear_q for M rows, K inputs and N
+ * outputs (INT8 rows, scales, row sums and the INT32 accumulators); 0 if
+ * M < 0, K < 1 or N < 1. */
+W4A8_API size_t w4z_workspace_size(int M, int K, int N);
+
+/*
+ * w4z_linear - the zero-point layer on float32 activations: activation pass,
+ * row sums, the W4A8 product on the stored codes, the zero-point epilogue
+ * (four launches). Arguments, flags and errors as for w4a8_linear, with
+ * sa/zp from w4z_quantize_pack in place of sw and a workspace of at least
+ * w4z_workspace_size(M, K, N) bytes.
+ */
+W4A8_API w4a8_status w4z_linear(const float *X, int M, int K, int ldx,
+                       const uint8_t *Wp, int ldp, const float *sa, const int32_t *zp, int N,
+                       const float *bias, unsigned flags, void *Y, int ldy,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* w4z_linear_q - the same on INT8 activations Xq [M][ldq] with scales sx [M]
+ * (three launches; the workspace holds the row sums and accumulators). */
+W4A8_API w4a8_status w4z_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                         const uint8_t *Wp, int ldp, const float *sa, const int32_t *zp, int N,
+                         const float *bias, unsigned flags, void *Y, int ldy,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
 /* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
  * last successful w4a8_linear / w4a8_linear_q / w8a8_linear / w8a8_linear_q
  * call enqueued (grouped calls: _DECODE); 0 if none. */

@@ -50,6 +50,11 @@ __device__ __forceinline__ uint32_t ld_dep_u8(const uint8_t *p) {
     asm volatile("ld.global.u8 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
+__device__ __forceinline__ int32_t ld_dep_s32(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.global.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ int32_t ld_dep_s8(const int8_t *p) {
     int32_t v;
     asm volatile("ld.global.s8 %0, [%1];" : "=r"(v) : "l"(p));

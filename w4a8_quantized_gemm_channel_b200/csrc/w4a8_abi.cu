@@ -12,6 +12,7 @@
 #include "quant_kernels.cuh"
 #include "linear_simt.cuh"
 #include "linear_w8.cuh"
+#include "zero_point.cuh"
 #include "decode_bulk.cuh"
 #include "gemm_tc.cuh"
 
@@ -329,6 +330,53 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     return W4A8_OK;
 }
 
+// -------------------------------------------------------- zero-point INT4 ---
+// Workspace of the zero-point calls: the INT8 rows and scales (w4z_linear
+// only), the row sums of the INT8 rows, and the INT32 accumulators of the
+// unchanged W4A8 product on the q - 8 codes.
+struct ZWorkspace {
+    Workspace a;
+    int *rowsum;
+    int32_t *acc;
+};
+
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+size_t zworkspace_bytes(int M, int K, int N) {
+    const int ldq = round_up(K, 16);
+    return round256((size_t)M * (size_t)ldq) + 2 * round256(sizeof(float) * (size_t)M) +
+           round256(sizeof(int32_t) * (size_t)M * (size_t)N) + 256;
+}
+
+ZWorkspace carve_zworkspace(void *ws, int M, int K) {
+    ZWorkspace z;
+    z.a = carve_workspace(ws, M, K);
+    uintptr_t p = reinterpret_cast<uintptr_t>(z.a.sx) + round256(sizeof(float) * (size_t)M);
+    z.rowsum = reinterpret_cast<int *>(p);
+    p += round256(sizeof(int) * (size_t)M);
+    z.acc = reinterpret_cast<int32_t *>(p);
+    return z;
+}
+
+// Row sums, the product on the q - 8 codes into the workspace, the
+// zero-point epilogue. after_act_pass: as for run_product.
+w4a8_status run_product_z(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
+                          const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
+                          int ldy, const ZWorkspace &zw, cudaStream_t s, bool after_act_pass) {
+    const int rows = M < 65535 ? M : 65535;
+    cudaError_t e = launch_pdl(zpt::k_row_sum8, dim3(rows), dim3(256), 0, s, Xq, M, K, ldq, zw.rowsum);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    const unsigned pflags = W4A8_OUT_S32 | (flags & (W4A8_PATH_MASK | W4A8_STATIC_WEIGHTS));
+    // the row-sum kernel waits before it lets dependents start, so the
+    // product may treat the weights as final exactly as behind the activation pass
+    w4a8_status st = run_product(Xq, M, K, ldq, sx, Wp, ldp, sa, N, nullptr, pflags, zw.acc, N, s, false,
+                                 after_act_pass);
+    if (st != W4A8_OK) return st;
+    e = launch_pdl(zpt::k_zp_epilogue, dim3((N + 255) / 256, rows), dim3(256), 0, s, zw.acc, M, N, zw.rowsum, zp,
+                   sx, sa, bias, flags, Y, ldy);
+    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ W8A8 ---
 // The INT8 path the INT4 steps extend: one INT8 weight code per byte, rows
 // of ldw8 >= K bytes (a multiple of 16), the same argument rules otherwise.
@@ -540,6 +588,40 @@ w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp,
 
 int w8a8_ld(int K) { return K < 1 ? -1 : round_up(K, 16); }
 
+size_t w4z_workspace_size(int M, int K, int N) {
+    if (M < 0 || K < 1 || N < 1) return 0;
+    return zworkspace_bytes(M, K, N);
+}
+
+w4a8_status w4z_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp, int ldp, float *sa, int32_t *zp,
+                              void *stream) {
+    if (!W || !Wp || !sa || !zp || K < 1 || K > W4A8_MAX_K || N < 1 || ldw < N) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(Wp) || ldp < (K + 1) / 2 || ldp % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (!aligned4(W) || !aligned4(sa) || !aligned4(zp)) return W4A8_ERR_INVALID_ARG;
+    const DeviceInfo &dev = device_info();
+    if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *lo = reinterpret_cast<int *>(zp), *hi = reinterpret_cast<int *>(sa);
+    zpt::k_minmax_init<<<(N + 255) / 256, 256, 0, s>>>(lo, hi, N);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    const int col_blocks = (N + 31) / 32;
+    int splits = (6 * dev.sm_count + col_blocks - 1) / col_blocks;
+    splits = splits < 1 ? 1 : splits;
+    int rows = (K + splits - 1) / splits;
+    rows = rows < 64 ? 64 : rows;
+    splits = (K + rows - 1) / rows;
+    if (splits > 65535) return W4A8_ERR_UNSUPPORTED;
+    zpt::k_col_minmax<<<dim3(col_blocks, splits), 256, 0, s>>>(W, K, N, ldw, rows, lo, hi);
+    if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
+    zpt::k_zp_finalize<<<(N + 255) / 256, 256, 0, s>>>(lo, hi, N);
+    if ((e = cudaGetLastError()) != cudaSuccess) return W4A8_ERR_CUDA;
+    const int kblocks = (2 * ldp + 63) / 64;
+    if (kblocks > 65535) return W4A8_ERR_UNSUPPORTED;
+    zpt::k_quant_pack_z<<<dim3(col_blocks, kblocks), 256, 0, s>>>(W, K, N, ldw, sa, zp, Wp, ldp);
+    return from_cuda(cudaGetLastError());
+}
+
 w4a8_status w8_quantize(const float *W, int K, int N, int ldw, int8_t *Wq, int ldw8, float *sw, void *stream) {
     if (!W || !Wq || !sw || K < 1 || K > W8A8_MAX_K || N < 1 || ldw < N) return W4A8_ERR_INVALID_ARG;
     if (!aligned16(Wq) || ldw8 < K || ldw8 % 16 != 0) return W4A8_ERR_INVALID_ARG;
@@ -705,6 +787,44 @@ w4a8_status w8a8_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *
     if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
     return run_product8(Xq, M, K, ldq, sx, Wq, ldw8, sw, N, bias, flags, Y, ldy,
                         static_cast<cudaStream_t>(stream));
+}
+
+w4a8_status w4z_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp, const float *sa,
+                       const int32_t *zp, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sa, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (!zp || !aligned4(zp) || ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    if (workspace_bytes < w4z_workspace_size(M, K, N)) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    const ZWorkspace zw = carve_zworkspace(workspace, M, K);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_act_quant(X, M, K, ldx, zw.a.xq, zw.a.ldq, zw.a.sx, s);
+    if (st != W4A8_OK) return st;
+    st = run_product_z(zw.a.xq, M, K, zw.a.ldq, zw.a.sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, zw, s, true);
+    if (st == W4A8_OK) t_last_launches = 4;
+    return st;
+}
+
+w4a8_status w4z_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
+                         const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
+                         int ldy, void *workspace, size_t workspace_bytes, void *stream) {
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sa, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (!zp || !aligned4(zp) || ldq < K || ldq % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    if (workspace_bytes < w4z_workspace_size(M, K, N)) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    const ZWorkspace zw = carve_zworkspace(workspace, M, K);
+    st = run_product_z(Xq, M, K, ldq, sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, zw,
+                       static_cast<cudaStream_t>(stream), false);
+    if (st == W4A8_OK) t_last_launches = 3;
+    return st;
 }
 
 unsigned w4a8_last_path(void) { return t_last_path; }

@@ -51,6 +51,10 @@ SIGNATURES = {
     "w8_quantize": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     "w8a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
     "w8a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
+    "w4z_quantize_pack": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P]),
+    "w4z_workspace_size": (_S, [_I, _I, _I]),
+    "w4z_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
+    "w4z_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
     "w4a8_last_path": (_U, []),
     "w4a8_last_launch_count": (_U, []),
     "w4a8_last_kernel": (ctypes.c_char_p, []),
@@ -296,6 +300,65 @@ def w8a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wq: torch.Tensor,
                              _ptr(bias), flags_for(relu, out, path, static_weights), _ptr(y), ldy,
                              _stream(stream)),
            "w8a8_linear_q")
+    return y
+
+
+# --------------------------------------------------- zero-point INT4 ---
+# Asymmetric per-channel INT4 weights (scale 15 / range, integer zero point),
+# stored as q - 8 nibbles in the W4A8 packed layout.
+
+def w4z_quantize_pack(w: torch.Tensor, stream=None):
+    """W[K][N] float32 (CUDA) -> (Wp[N][ldp] uint8, sa[N] float32, zp[N] int32)."""
+    ldw = _rowmajor(w, "W")
+    k, n = w.shape
+    wp = torch.empty((n, packed_ld(k)), dtype=torch.uint8, device=w.device)
+    sa = torch.empty(n, dtype=torch.float32, device=w.device)
+    zp = torch.empty(n, dtype=torch.int32, device=w.device)
+    _check(lib.w4z_quantize_pack(_ptr(w), k, n, ldw, _ptr(wp), wp.stride(0), _ptr(sa), _ptr(zp),
+                                 _stream(stream)), "w4z_quantize_pack")
+    return wp, sa, zp
+
+
+def _zworkspace(workspace, m, k, n, device):
+    need = lib.w4z_workspace_size(m, k, n)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def w4z_linear(x: torch.Tensor, wp: torch.Tensor, sa: torch.Tensor, zp: torch.Tensor,
+               bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
+               path: str = "auto", y: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None,
+               static_weights: bool = False) -> torch.Tensor:
+    """Y[M][N] of the zero-point layer for X[M][K] float32."""
+    ldx = _rowmajor(x, "X")
+    ldp = _rowmajor(wp, "Wp")
+    m, k = x.shape
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, x.device)
+    workspace, wsb = _zworkspace(workspace, m, k, n, x.device)
+    _check(lib.w4z_linear(_ptr(x), m, k, ldx, _ptr(wp), ldp, _ptr(sa), _ptr(zp), n, _ptr(bias),
+                          flags_for(relu, out, path, static_weights), _ptr(y), ldy, _ptr(workspace), wsb,
+                          _stream(stream)), "w4z_linear")
+    return y
+
+
+def w4z_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor, sa: torch.Tensor,
+                 zp: torch.Tensor, bias: torch.Tensor | None = None, relu: bool = False,
+                 out: str = "f32", path: str = "auto", y: torch.Tensor | None = None,
+                 workspace: torch.Tensor | None = None, stream=None,
+                 static_weights: bool = False) -> torch.Tensor:
+    """The zero-point layer on INT8 activations Xq[M][ldq] and sx[M]."""
+    ldq = _rowmajor(xq, "Xq")
+    ldp = _rowmajor(wp, "Wp")
+    m = xq.shape[0]
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, xq.device)
+    workspace, wsb = _zworkspace(workspace, m, k, n, xq.device)
+    _check(lib.w4z_linear_q(_ptr(xq), m, k, ldq, _ptr(sx), _ptr(wp), ldp, _ptr(sa), _ptr(zp), n, _ptr(bias),
+                            flags_for(relu, out, path, static_weights), _ptr(y), ldy, _ptr(workspace), wsb,
+                            _stream(stream)), "w4z_linear_q")
     return y
 
 
