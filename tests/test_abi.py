@@ -167,3 +167,32 @@ def test_grouped_rejects_bad_arguments_before_the_device():
     arr = (P * 1)(P(16, 4096, 8192, None, 12288, 2, 64, 64, 32, 8, 8))
     assert native.lib.w4a8_linear_grouped(arr, 1, native.PATH_TC, None) == native.ERR_INVALID_ARG
     assert ct.sizeof(P) == 64
+
+
+def test_zero_point_calls_check_arguments_before_the_device():
+    """The zero-point entry points reject bad arguments (and report the
+    workspace size) without touching a device."""
+    from w4a8_quantized_gemm_channel_b200 import native
+    lib = native.lib
+    m, k, n = 4, 64, 8
+    need = lib.w4z_workspace_size(m, k, n)
+    # INT8 rows + scales + row sums + INT32 accumulators, each 256-aligned, + slack
+    assert need >= m * 64 + 4 * m + 4 * m + 4 * m * n
+    assert lib.w4z_workspace_size(-1, k, n) == 0 and lib.w4z_workspace_size(m, 0, n) == 0
+    assert lib.w4z_workspace_size(m, k, 0) == 0
+    args = dict(X=16, M=m, K=k, ldx=k, Wp=4096, ldp=32, sa=8192, zp=8448, N=n, bias=None, flags=0,
+                Y=12288, ldy=n, ws=16384, wsb=need, stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.w4z_linear(a["X"], a["M"], a["K"], a["ldx"], a["Wp"], a["ldp"], a["sa"], a["zp"], a["N"],
+                              a["bias"], a["flags"], a["Y"], a["ldy"], a["ws"], a["wsb"], a["stream"])
+    assert call(zp=None) == 1            # zero points missing
+    assert call(zp=8450) == 1            # misaligned zero points
+    assert call(ldp=16) == 1             # ldp < ceil(K/2)
+    assert call(K=0) == 1
+    assert call(ws=None) == 3 and call(wsb=need - 1) == 3
+    assert call(M=0) == 0                # no rows: a no-op
+    assert lib.w4z_quantize_pack(16, k, n, n, 4096, 32, 64, None, None) == 1   # zp missing
+    assert lib.w4z_quantize_pack(16, k, n, n - 1, 4096, 32, 64, 128, None) == 1  # ldw < N
+    assert lib.w4z_linear_q(24, 2, k, k, 64, 4096, 32, 64, 128, n, None, 0, 8192, n, 16384, need, None) == 1
