@@ -69,6 +69,8 @@ def _load():
                 "oracle_gemm8_s32": [P, I, I, I, P, I, I, P, I],
                 "oracle_w4z_quantize_pack": [P, I, I, I, P, I, P, P],
                 "oracle_gemm_z_s32": [P, I, I, I, P, I, I, P, P, I],
+                "oracle_w4g_quantize_pack": [P, I, I, I, I, P, I, P, P],
+                "oracle_linear_g_q": [P, P, I, I, I, P, I, I, I, P, P, P, I, P, P, I],
             }.items():
                 fn = getattr(lib, name)
                 fn.argtypes = args
@@ -311,6 +313,43 @@ def linear_z(x: np.ndarray, wp: np.ndarray, sa: np.ndarray, zp: np.ndarray, k: i
         return acc
     y = dequant(acc, sx, sa, bias, relu)
     return to_bf16_bits(y) if out == "bf16" else y
+
+
+# ---------------------------------------------------- group-wise INT4 ---
+# "INT4" concept page, section 4.2: every group of G consecutive k of an
+# output channel has its own scale and zero point (the zero-point rule above
+# per group); partial INT32 sums per group, dequantized per group and summed
+# over the groups in float32.
+
+def w4g_quantize_pack(w: np.ndarray, group: int, ldp: int | None = None):
+    """W[K][N] float32 -> (Wp[N][ldp] uint8, sa[N][ng] float32, zp[N][ng] int32)."""
+    w = _f32(w)
+    k, n = w.shape
+    ng = -(-k // group)
+    ldp = packed_ld(k) if ldp is None else ldp
+    wp = np.empty((n, ldp), np.uint8)
+    sa = np.empty((n, ng), np.float32)
+    zp = np.empty((n, ng), np.int32)
+    _check(_load().oracle_w4g_quantize_pack(_ptr(w), k, n, n, group, _ptr(wp), ldp, _ptr(sa), _ptr(zp)),
+           "w4g_quantize_pack")
+    return wp, sa, zp
+
+
+def linear_g(x: np.ndarray, wp: np.ndarray, sa: np.ndarray, zp: np.ndarray, k: int, group: int,
+             bias: np.ndarray | None = None, relu: bool = False, partials: bool = False):
+    """One group-wise INT4 Dense layer on float32 input; with partials=True
+    also returns the INT32 partial sums [M][N][ng]."""
+    xq, sx = a8_quantize_rows(x)
+    m = xq.shape[0]
+    n, ldp = wp.shape
+    ng = sa.shape[1]
+    acc_g = np.empty((m, n, ng), np.int32)
+    y = np.empty((m, n), np.float32)
+    b = None if bias is None else _f32(bias)
+    _check(_load().oracle_linear_g_q(_ptr(xq), _ptr(sx), m, k, xq.shape[1], _ptr(np.ascontiguousarray(wp)), n,
+                                     ldp, group, _ptr(_f32(sa)), _ptr(np.ascontiguousarray(zp, np.int32)), _ptr(b),
+                                     int(bool(relu)), _ptr(acc_g), _ptr(y), n), "linear_g")
+    return (y, acc_g) if partials else y
 
 
 def mlp(x: np.ndarray, w1, b1, w2, b2) -> np.ndarray:

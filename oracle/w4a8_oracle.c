@@ -41,6 +41,16 @@
  * per byte along K, even k in the low nibble; the product
  * acc = sum_k xq * (q - zp) and y = float(acc) / (sx * sa).
  *
+ * Group-wise INT4 (the "INT4" concept page, section 4.2, group quantization:
+ * each group of group_size weights along the input axis, e.g. 128, has its own
+ * scale and zero point; the "4-bit Integer Quantization for LLMs" page's
+ * quantization configuration names group_size 128): read as the zero-point
+ * rule above applied to every (output channel n, group g of G consecutive k)
+ * separately, the last group ragged when G does not divide K. The product is
+ * the INT32 partial sum of each group, dequantized by its own scale and
+ * summed over the groups in increasing g in float32:
+ *   y = sum_g float(sum_{k in g} xq * (q - zp[n][g])) / (sx * sa[n][g]).
+ *
  * Precision: the page's model is float32 end to end (its inputs are cast with
  * astype("float32")), and float32 decides every integer code, so each step
  * below runs in float32 with IEEE round-to-nearest. Build flags:
@@ -378,6 +388,80 @@ int oracle_gemm_z_s32(const int8_t *Xq, int M, int K, int ldq, const uint8_t *Wp
                 s += (int64_t)Xq[(size_t)m * ldq + k] * (int64_t)(zp_code(Wp, ldp, n, k) - zp[n]);
             if (s > INT32_MAX || s < INT32_MIN) return ORACLE_OVERFLOW;
             acc[(size_t)m * ldacc + n] = (int32_t)s;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Group-wise INT4: the zero-point rule per (output channel n, group g of G
+ * consecutive k; the last group holds K - G * (ng - 1) of them), ng =
+ * ceil(K / G). sa, zp are [N][ng]. Codes packed as for the zero-point form
+ * (unsigned nibbles, even k low, zero pad).
+ * ------------------------------------------------------------------------- */
+int oracle_w4g_quantize_pack(const float *W, int K, int N, int ldw, int G, uint8_t *Wp, int ldp,
+                             float *sa, int32_t *zp)
+{
+    if (!W || !Wp || !sa || !zp || K < 1 || N < 1 || G < 1 || ldw < N || ldp < (K + 1) / 2) return ORACLE_BAD_ARG;
+    const int ng = (K + G - 1) / G;
+    for (int n = 0; n < N; ++n) {
+        uint8_t *row = Wp + (size_t)n * ldp;
+        memset(row, 0, (size_t)ldp);
+        for (int g = 0; g < ng; ++g) {
+            const int k0 = g * G, k1 = (k0 + G < K) ? k0 + G : K;
+            float lo = W[(size_t)k0 * ldw + n], hi = lo;
+            for (int k = k0 + 1; k < k1; ++k) {
+                float w = W[(size_t)k * ldw + n];
+                if (w < lo) lo = w;
+                if (w > hi) hi = w;
+            }
+            float range = hi - lo;
+            float s = (range == 0.0f) ? 1.0f : 15.0f / range;
+            int32_t z = -(int32_t)round_half_even(lo * s);
+            sa[(size_t)n * ng + g] = s;
+            zp[(size_t)n * ng + g] = z;
+            for (int k = k0; k < k1; ++k) {
+                float t = W[(size_t)k * ldw + n] * s;
+                int q = clamp_int((int)round_half_even(t) + z, 0, 15);
+                if (k % 2 == 0)
+                    row[k / 2] |= (uint8_t)q;
+                else
+                    row[k / 2] |= (uint8_t)(q << 4);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Group-wise product: per (m, n) the INT32 partial sum of each group (exact,
+ * int64, required to fit INT32), dequantized by that group's scale and the
+ * row scale, summed over increasing g in float32; then bias and ReLU as in
+ * oracle_dequant. acc_g (M * N * ng int32) receives the partial sums. */
+int oracle_linear_g_q(const int8_t *Xq, const float *sx, int M, int K, int ldq, const uint8_t *Wp, int N,
+                      int ldp, int G, const float *sa, const int32_t *zp, const float *bias, int relu,
+                      int32_t *acc_g, float *Y, int ldy)
+{
+    if (M < 0 || K < 1 || N < 1 || G < 1 || ldq < K || ldp < (K + 1) / 2 || ldy < N) return ORACLE_BAD_ARG;
+    if (M == 0) return ORACLE_OK;
+    if (!Xq || !sx || !Wp || !sa || !zp || !acc_g || !Y) return ORACLE_BAD_ARG;
+    const int ng = (K + G - 1) / G;
+    for (int m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            float y = 0.0f;
+            for (int g = 0; g < ng; ++g) {
+                const int k0 = g * G, k1 = (k0 + G < K) ? k0 + G : K;
+                int64_t s = 0;
+                for (int k = k0; k < k1; ++k)
+                    s += (int64_t)Xq[(size_t)m * ldq + k] *
+                         (int64_t)(zp_code(Wp, ldp, n, k) - zp[(size_t)n * ng + g]);
+                if (s > INT32_MAX || s < INT32_MIN) return ORACLE_OVERFLOW;
+                acc_g[((size_t)m * N + n) * ng + g] = (int32_t)s;
+                float d = sx[m] * sa[(size_t)n * ng + g];
+                y = y + (float)s / d;
+            }
+            if (bias) y = y + bias[n];
+            if (relu) y = (y > 0.0f) ? y : 0.0f;
+            Y[(size_t)m * ldy + n] = y;
         }
     }
     return ORACLE_OK;

@@ -530,3 +530,93 @@ def test_linear_z_error_bound_and_tighter_than_symmetric():
     wps, sws = oracle.w4_quantize_pack(w)
     ys = oracle.linear(x, wps, sws, 640)
     assert np.abs(y - exact).mean() < np.abs(ys - exact).mean()
+
+
+# ---------------------------------------------------- group-wise INT4 ---
+# "INT4" concept page, section 4.2 (group quantization: each group of
+# group_size weights has its own scale and zero point).
+
+def test_w4g_hand_worked_two_groups():
+    """K = 6, G = 4: group 0 = [-1, 0, 2, 0.5] -> sa 5, zp 5, codes 0 5 15 7;
+    group 1 = [10, 20] (ragged) -> sa 15/10 = 1.5, zp -rne(15) = -15, codes 0, 15.
+    With X = ones (sx = 127, codes 127) the partial sums are 127 * 7 = 889 and
+    127 * 45 = 5715, and y = fl(fl(889 / 635) + fl(5715 / 190.5))."""
+    w = np.array([[-1.0], [0.0], [2.0], [0.5], [10.0], [20.0]], np.float32)
+    wp, sa, zp = oracle.w4g_quantize_pack(w, 4)
+    assert sa.tolist() == [[5.0, 1.5]] and zp.tolist() == [[5, -15]]
+    assert wp[0, :3].tolist() == [80, 127, 240] and not wp[0, 3:].any()
+    y, acc = oracle.linear_g(np.ones((1, 6), np.float32), wp, sa, zp, 6, 4, partials=True)
+    assert acc.tolist() == [[[889, 5715]]]
+    f = np.float32
+    assert y[0, 0] == f(f(f(889) / f(635)) + f(f(5715) / f(190.5)))
+
+
+def test_w4g_one_group_is_the_per_channel_zero_point_layer():
+    """G >= K leaves one group per channel: codes, scales, zero points,
+    accumulators and outputs are those of the per-channel zero-point layer."""
+    x, _ = synth.linear_activations(5, 300, seed=51, outlier_count=3, outlier_factor=20.0)
+    w = synth.linear_weights(300, 24, 0.02, seed=51)
+    b = synth.bias_vector(24, 51)
+    wpz, saz, zpz = oracle.w4z_quantize_pack(w)
+    for g in (300, 512):
+        wp, sa, zp = oracle.w4g_quantize_pack(w, g)
+        assert np.array_equal(wp, wpz) and np.array_equal(sa[:, 0], saz) and np.array_equal(zp[:, 0], zpz)
+        y, acc = oracle.linear_g(x, wp, sa, zp, 300, g, bias=b, relu=True, partials=True)
+        assert np.array_equal(acc[:, :, 0], oracle.linear_z(x, wpz, saz, zpz, 300, out="s32"))
+        assert np.array_equal(y, oracle.linear_z(x, wpz, saz, zpz, 300, bias=b, relu=True))
+
+
+def test_w4g_groups_are_independent_and_dequantize_within_a_step():
+    """Changing the weights of one group changes no other group's codes or
+    scales; every weight dequantizes within 1 / sa of its group."""
+    k, n, G = 640, 16, 128
+    w = _random_w(k=k, n=n, seed=52)
+    wp, sa, zp = oracle.w4g_quantize_pack(w, G)
+    w2 = w.copy()
+    w2[256:384] *= np.float32(3.0)  # group 2 only
+    wp2, sa2, zp2 = oracle.w4g_quantize_pack(w2, G)
+    q = _unpack_unsigned(wp, k)
+    q2 = _unpack_unsigned(wp2, k)
+    others = np.r_[0:256, 384:640]
+    assert np.array_equal(q[:, others], q2[:, others])
+    assert np.array_equal(np.delete(sa, 2, axis=1), np.delete(sa2, 2, axis=1))
+    assert np.array_equal(np.delete(zp, 2, axis=1), np.delete(zp2, 2, axis=1))
+    g_of_k = np.arange(k) // G
+    deq = (q - zp[:, g_of_k].astype(np.int64)) / sa[:, g_of_k].astype(np.float64)
+    assert (np.abs(w.T.astype(np.float64) - deq) <= (1.0 / sa[:, g_of_k].astype(np.float64)) * (1 + 1e-6)).all()
+
+
+def test_w4g_output_is_the_float32_sum_of_group_terms():
+    """y against the float64 sum of the same per-group terms (from the INT32
+    partials): float32 rounding of ng quotients and ng additions stays within
+    (2 ng + 2) * 2^-24 of the sum of |terms|; and the partials sum to an exact
+    float64 matmul of the dequantization-free integer form."""
+    k, n, G = 1000, 20, 128
+    x, _ = synth.linear_activations(6, k, seed=53, outlier_count=4, outlier_factor=20.0)
+    w = synth.linear_weights(k, n, 0.02, seed=53)
+    wp, sa, zp = oracle.w4g_quantize_pack(w, G)
+    y, acc = oracle.linear_g(x, wp, sa, zp, k, G, partials=True)
+    xq, sx = oracle.a8_quantize_rows(x)
+    ng = sa.shape[1]
+    terms = acc.astype(np.float64) / (sx.astype(np.float64)[:, None, None] * sa.astype(np.float64)[None, :, :])
+    ref = terms.sum(axis=2)
+    tol = (2 * ng + 2) * 2.0 ** -24 * np.abs(terms).sum(axis=2)
+    assert (np.abs(y - ref) <= tol).all()
+    q = _unpack_unsigned(wp, k) - zp[:, np.arange(k) // G].astype(np.int64)
+    for g in range(ng):
+        ks = slice(g * G, min(k, (g + 1) * G))
+        assert np.array_equal(acc[:, :, g].astype(np.float64),
+                              xq[:, ks].astype(np.float64) @ q[:, ks].T.astype(np.float64))
+
+
+def test_w4g_error_below_per_channel_zero_point():
+    """Finer groups, finer grids: on the same data the group-wise layer's mean
+    error against X @ W is below the per-channel zero-point layer's."""
+    x, _ = synth.linear_activations(8, 1024, seed=54, outlier_count=3, outlier_factor=20.0)
+    w = synth.linear_weights(1024, 48, 0.02, seed=54)
+    exact = x.astype(np.float64) @ w.astype(np.float64)
+    wp, sa, zp = oracle.w4g_quantize_pack(w, 128)
+    yg = oracle.linear_g(x, wp, sa, zp, 1024, 128)
+    wpz, saz, zpz = oracle.w4z_quantize_pack(w)
+    yz = oracle.linear_z(x, wpz, saz, zpz, 1024)
+    assert np.abs(yg - exact).mean() < np.abs(yz - exact).mean()
