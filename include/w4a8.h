@@ -315,6 +315,42 @@ W4A8_API w4a8_status w4z_linear_q(const int8_t *Xq, int M, int K, int ldq, const
                          const float *bias, unsigned flags, void *Y, int ldy,
                          void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Group-wise INT4 - the zero-point rule above applied to every group of 128
+ * consecutive k of each output channel ("INT4" concept page, section 4.2,
+ * group quantization with group_size 128); sa and zp are [N][ng] with
+ * ng = ceil(K / 128), the last group ragged. The output is
+ *   y = sum_g float(acc_g) / (sx[m] * sa[n][g]),
+ *   acc_g = sum_{k in g} xq[m][k] * (q - zp[n][g]) (exact INT32 partial sums),
+ * summed in float32, then bias and ReLU. The kernel adds the group terms in
+ * another order than a sequential loop, so outputs agree with that loop
+ * within (2 ng + 2) * 2^-24 * sum_g |term_g| rather than bit for bit.
+ * Storage: as for the zero-point form (nibbles q - 8, pad 0).
+ * Output formats: W4A8_OUT_F32 or _BF16 (W4A8_OUT_S32 is rejected: there is no
+ * single integer accumulator). Path: the decode-style kernel for any M
+ * (W4A8_PATH_AUTO or _DECODE; other paths return W4A8_ERR_UNSUPPORTED).
+ */
+
+/* Groups per output channel for K inputs: ceil(K / 128); -1 if K < 1. */
+W4A8_API int w4g_groups(int K);
+
+/* w4g_quantize_pack - W [K][ldw] float32 -> Wp [N][ldp] (as w4z_quantize_pack),
+ * sa [N][ng] float32, zp [N][ng] int32. Requires 1 <= K <= W4A8_MAX_K, N >= 1. */
+W4A8_API w4a8_status w4g_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp, int ldp,
+                              float *sa, int32_t *zp, void *stream);
+
+/* w4g_linear - activation pass and the group-wise product (two launches);
+ * arguments and workspace (w4a8_workspace_size(M, K)) as for w4a8_linear. */
+W4A8_API w4a8_status w4g_linear(const float *X, int M, int K, int ldx,
+                       const uint8_t *Wp, int ldp, const float *sa, const int32_t *zp, int N,
+                       const float *bias, unsigned flags, void *Y, int ldy,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* w4g_linear_q - the group-wise product on INT8 activations (one launch). */
+W4A8_API w4a8_status w4g_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
+                         const uint8_t *Wp, int ldp, const float *sa, const int32_t *zp, int N,
+                         const float *bias, unsigned flags, void *Y, int ldy, void *stream);
+
 /* Which kernel path (W4A8_PATH_GENERIC / _DECODE / _TC) the calling thread's
  * last successful w4a8_linear / w4a8_linear_q / w8a8_linear / w8a8_linear_q
  * call enqueued (grouped calls: _DECODE); 0 if none. */

@@ -196,3 +196,22 @@ def test_zero_point_calls_check_arguments_before_the_device():
     assert lib.w4z_quantize_pack(16, k, n, n, 4096, 32, 64, None, None) == 1   # zp missing
     assert lib.w4z_quantize_pack(16, k, n, n - 1, 4096, 32, 64, 128, None) == 1  # ldw < N
     assert lib.w4z_linear_q(24, 2, k, k, 64, 4096, 32, 64, 128, n, None, 0, 8192, n, 16384, need, None) == 1
+
+
+def test_group_wise_calls_check_arguments_before_the_device():
+    from w4a8_quantized_gemm_channel_b200 import native
+    lib = native.lib
+    assert lib.w4g_groups(1) == 1 and lib.w4g_groups(128) == 1 and lib.w4g_groups(129) == 2
+    assert lib.w4g_groups(0) == -1
+    m, k, n = 4, 300, 8
+    a = dict(X=16, M=m, K=k, ldx=k, Wp=4096, ldp=160, sa=8192, zp=8448, N=n, bias=None, flags=0,
+             Y=12288, ldy=n, ws=16384, wsb=1 << 20, stream=None)
+
+    def call(**kw):
+        b = dict(a, **kw)
+        return lib.w4g_linear(b["X"], b["M"], b["K"], b["ldx"], b["Wp"], b["ldp"], b["sa"], b["zp"], b["N"],
+                              b["bias"], b["flags"], b["Y"], b["ldy"], b["ws"], b["wsb"], b["stream"])
+    assert call(flags=0x04) == 1      # INT32 output: no single accumulator in this form
+    assert call(zp=None) == 1 and call(ldp=144) == 1 and call(ws=None) == 3
+    assert call(M=0) == 0
+    assert lib.w4g_quantize_pack(16, k, n, n, 4096, 160, 64, None, None) == 1

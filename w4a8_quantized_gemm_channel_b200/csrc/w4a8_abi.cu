@@ -13,6 +13,7 @@
 #include "linear_simt.cuh"
 #include "linear_w8.cuh"
 #include "zero_point.cuh"
+#include "group_wise.cuh"
 #include "decode_bulk.cuh"
 #include "gemm_tc.cuh"
 
@@ -377,6 +378,29 @@ w4a8_status run_product_z(const int8_t *Xq, int M, int K, int ldq, const float *
     return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
+// ------------------------------------------------------- group-wise INT4 ---
+// The group-wise product (any M, tiles of 8 or 16 tokens; float32 outputs).
+w4a8_status run_product_g(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
+                          const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
+                          int ldy, cudaStream_t stream, bool after_act_pass) {
+    const unsigned path = flags & W4A8_PATH_MASK;
+    if (path != W4A8_PATH_AUTO && path != W4A8_PATH_DECODE) return W4A8_ERR_UNSUPPORTED;
+    const int tok = M <= 8 ? 8 : 16;
+    const int tiles = (M + tok - 1) / tok;
+    if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
+    dim3 grid((N + 15) / 16, tiles);
+    const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
+    auto kern = tok == 8 ? (early ? grp::k_linear_g<1, true> : grp::k_linear_g<1, false>)
+                         : (early ? grp::k_linear_g<2, true> : grp::k_linear_g<2, false>);
+    cudaError_t e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream, Xq, M, K, ldq, sx, Wp, ldp, sa, zp,
+                               grp::groups_of(K), N, bias, flags, Y, ldy);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    t_last_path = W4A8_PATH_DECODE;
+    t_last_launches = 1;
+    t_last_kernel = "k_linear_g";
+    return W4A8_OK;
+}
+
 // ------------------------------------------------------------------ W8A8 ---
 // The INT8 path the INT4 steps extend: one INT8 weight code per byte, rows
 // of ldw8 >= K bytes (a multiple of 16), the same argument rules otherwise.
@@ -587,6 +611,23 @@ w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp,
 }
 
 int w8a8_ld(int K) { return K < 1 ? -1 : round_up(K, 16); }
+
+int w4g_groups(int K) { return K < 1 ? -1 : grp::groups_of(K); }
+
+w4a8_status w4g_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp, int ldp, float *sa, int32_t *zp,
+                              void *stream) {
+    if (!W || !Wp || !sa || !zp || K < 1 || K > W4A8_MAX_K || N < 1 || ldw < N) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(Wp) || ldp < (K + 1) / 2 || ldp % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (!aligned4(W) || !aligned4(sa) || !aligned4(zp)) return W4A8_ERR_INVALID_ARG;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // every byte of every row, the parts no group covers included, starts at 0
+    cudaError_t e = cudaMemset2DAsync(Wp, (size_t)ldp, 0, (size_t)ldp, (size_t)N, s);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    const int ng = grp::groups_of(K);
+    grp::k_quant_pack_g<<<dim3((N + 127) / 128, ng), 128, 0, s>>>(W, K, N, ldw, Wp, ldp, sa, zp, ng);
+    return from_cuda(cudaGetLastError());
+}
 
 size_t w4z_workspace_size(int M, int K, int N) {
     if (M < 0 || K < 1 || N < 1) return 0;
@@ -825,6 +866,49 @@ w4a8_status w4z_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *s
                        static_cast<cudaStream_t>(stream), false);
     if (st == W4A8_OK) t_last_launches = 3;
     return st;
+}
+
+static w4a8_status check_g(int M, int K, int N, const uint8_t *Wp, int ldp, const float *sa, const int32_t *zp,
+                           const float *bias, unsigned flags, const void *Y, int ldy) {
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sa, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (!zp || !aligned4(zp)) return W4A8_ERR_INVALID_ARG;
+    // the output is a float sum over groups: there is no single INT32 accumulator
+    if ((flags & W4A8_OUT_MASK) == W4A8_OUT_S32) return W4A8_ERR_INVALID_ARG;
+    return W4A8_OK;
+}
+
+w4a8_status w4g_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp, int ldp, const float *sa,
+                       const int32_t *zp, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    w4a8_status st = check_g(M, K, N, Wp, ldp, sa, zp, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    if (workspace_bytes < w4a8_workspace_size(M, K)) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    const Workspace ws = carve_workspace(workspace, M, K);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
+    if (st != W4A8_OK) return st;
+    st = run_product_g(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, s, true);
+    if (st == W4A8_OK) t_last_launches = 2;
+    return st;
+}
+
+w4a8_status w4g_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
+                         const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
+                         int ldy, void *stream) {
+    w4a8_status st = check_g(M, K, N, Wp, ldp, sa, zp, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldq < K || ldq % 16 != 0) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!Xq || !sx || !aligned16(Xq) || !aligned4(sx)) return W4A8_ERR_INVALID_ARG;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    return run_product_g(Xq, M, K, ldq, sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy,
+                         static_cast<cudaStream_t>(stream), false);
 }
 
 unsigned w4a8_last_path(void) { return t_last_path; }

@@ -55,6 +55,10 @@ SIGNATURES = {
     "w4z_workspace_size": (_S, [_I, _I, _I]),
     "w4z_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
     "w4z_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
+    "w4g_groups": (_I, [_I]),
+    "w4g_quantize_pack": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P]),
+    "w4g_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
+    "w4g_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_last_path": (_U, []),
     "w4a8_last_launch_count": (_U, []),
     "w4a8_last_kernel": (ctypes.c_char_p, []),
@@ -359,6 +363,58 @@ def w4z_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor, s
     _check(lib.w4z_linear_q(_ptr(xq), m, k, ldq, _ptr(sx), _ptr(wp), ldp, _ptr(sa), _ptr(zp), n, _ptr(bias),
                             flags_for(relu, out, path, static_weights), _ptr(y), ldy, _ptr(workspace), wsb,
                             _stream(stream)), "w4z_linear_q")
+    return y
+
+
+# ---------------------------------------------------- group-wise INT4 ---
+# Per (output channel, group of 128 k) scale and zero point; float32 outputs.
+
+def w4g_quantize_pack(w: torch.Tensor, stream=None):
+    """W[K][N] float32 (CUDA) -> (Wp[N][ldp] uint8, sa[N][ng] float32, zp[N][ng] int32)."""
+    ldw = _rowmajor(w, "W")
+    k, n = w.shape
+    ng = lib.w4g_groups(k)
+    wp = torch.empty((n, packed_ld(k)), dtype=torch.uint8, device=w.device)
+    sa = torch.empty((n, ng), dtype=torch.float32, device=w.device)
+    zp = torch.empty((n, ng), dtype=torch.int32, device=w.device)
+    _check(lib.w4g_quantize_pack(_ptr(w), k, n, ldw, _ptr(wp), wp.stride(0), _ptr(sa), _ptr(zp),
+                                 _stream(stream)), "w4g_quantize_pack")
+    return wp, sa, zp
+
+
+def w4g_linear(x: torch.Tensor, wp: torch.Tensor, sa: torch.Tensor, zp: torch.Tensor,
+               bias: torch.Tensor | None = None, relu: bool = False, out: str = "f32",
+               path: str = "auto", y: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None,
+               static_weights: bool = False) -> torch.Tensor:
+    """Y[M][N] of the group-wise layer for X[M][K] float32."""
+    ldx = _rowmajor(x, "X")
+    ldp = _rowmajor(wp, "Wp")
+    m, k = x.shape
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, x.device)
+    need = workspace_size(m, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(lib.w4g_linear(_ptr(x), m, k, ldx, _ptr(wp), ldp, _ptr(sa), _ptr(zp), n, _ptr(bias),
+                          flags_for(relu, out, path, static_weights), _ptr(y), ldy, _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream)), "w4g_linear")
+    return y
+
+
+def w4g_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor, sa: torch.Tensor,
+                 zp: torch.Tensor, bias: torch.Tensor | None = None, relu: bool = False,
+                 out: str = "f32", path: str = "auto", y: torch.Tensor | None = None, stream=None,
+                 static_weights: bool = False) -> torch.Tensor:
+    """The group-wise layer on INT8 activations Xq[M][ldq] and sx[M]."""
+    ldq = _rowmajor(xq, "Xq")
+    ldp = _rowmajor(wp, "Wp")
+    m = xq.shape[0]
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, out, xq.device)
+    _check(lib.w4g_linear_q(_ptr(xq), m, k, ldq, _ptr(sx), _ptr(wp), ldp, _ptr(sa), _ptr(zp), n, _ptr(bias),
+                            flags_for(relu, out, path, static_weights), _ptr(y), ldy, _stream(stream)),
+           "w4g_linear_q")
     return y
 
 
