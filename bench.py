@@ -125,27 +125,30 @@ class DecodeWorkload:
     outlier channels x20."""
     name = "decode"
 
-    def __init__(self, torch, native, synth, device, l2_bytes, w8=False, zp=False):
+    def __init__(self, torch, native, synth, device, l2_bytes, w8=False, zp=False, grp=False):
         self.torch, self.nat = torch, native
         self.w8 = w8  # the W8A8 path: INT8 weight rows instead of packed INT4
         self.zpf = zp  # the zero-point INT4 path: asymmetric per-channel weights
+        self.grp = grp  # the group-wise INT4 path: scale and zero point per 128 weights
         self.K, self.N, self.MS = synth.DECODE_K, synth.DECODE_N, synth.DECODE_MS
         w = synth.decode_case(1).w
         self.w_host = w
         wd = torch.from_numpy(w).to(device)
-        if zp:
+        if grp:
+            wp, sw, zpt = native.w4g_quantize_pack(wd)
+        elif zp:
             wp, sw, zpt = native.w4z_quantize_pack(wd)
         else:
             wp, sw = native.w8_quantize(wd) if w8 else native.w4_quantize_pack(wd)
         self.wd = wd
-        per_weight = wp.numel() + 4 * sw.numel() * (2 if zp else 1)
+        per_weight = wp.numel() + 4 * sw.numel() * (2 if (zp or grp) else 1)
         # enough distinct copies (>= 3x L2) that each launch's weights were
         # evicted from L2 since their last use
         need = -(-3 * l2_bytes // per_weight) + len(self.MS)
         self.pool = -(-need // len(self.MS)) * len(self.MS)
         self.wp = [wp.clone() for _ in range(self.pool)]
         self.sw = [sw.clone() for _ in range(self.pool)]
-        self.zp = [zpt.clone() for _ in range(self.pool)] if zp else None
+        self.zp = [zpt.clone() for _ in range(self.pool)] if (zp or grp) else None
         self.x_host = {m: synth.decode_case(m).x for m in self.MS}
         self.x = {m: torch.from_numpy(self.x_host[m]).to(device) for m in self.MS}
         self.y = {m: torch.empty((m, self.N), dtype=torch.float32, device=device) for m in self.MS}
@@ -159,14 +162,17 @@ class DecodeWorkload:
         return self.nat.w8a8_ld(self.K) if self.w8 else self.nat.packed_ld(self.K)
 
     def linear_q(self, xq, sx, k, wp, sw, **kw):
-        if self.zpf:
+        if self.zpf or self.grp:
             i = next(j for j, t in enumerate(self.wp) if t is wp)
+            if self.grp:
+                return self.nat.w4g_linear_q(xq, sx, k, wp, sw, self.zp[i], **kw)
             return self.nat.w4z_linear_q(xq, sx, k, wp, sw, self.zp[i], workspace=self.ws[xq.shape[0]], **kw)
         return (self.nat.w8a8_linear_q if self.w8 else self.nat.w4a8_linear_q)(xq, sx, k, wp, sw, **kw)
 
     def bytes_per_step(self):
         ldp = self.weight_ld()
-        scales = (8 if self.zpf else 4) * self.N
+        # scales (and zero points) per launch: sw [N]; zero-point: + zp [N]; group-wise: sa, zp [N][ng]
+        scales = 8 * self.N if self.zpf else (8 * self.sw[0].numel() if self.grp else 4 * self.N)
         return sum(self.N * ldp + scales + 4 * m * self.K + 4 * m * self.N for m in self.MS)
 
     def ops_per_step(self):
@@ -185,6 +191,10 @@ class DecodeWorkload:
         # weights were quantized before timing and the stream has synchronized
         # since: the serving-style call promises they are settled
         xx = self.x[m] if x is None else x
+        if self.grp:
+            self.nat.w4g_linear(xx, self.wp[s], self.sw[s], self.zp[s], y=self.y[m], workspace=self.ws[m],
+                                static_weights=True)
+            return
         if self.zpf:
             self.nat.w4z_linear(xx, self.wp[s], self.sw[s], self.zp[s], y=self.y[m], workspace=self.ws[m],
                                 static_weights=True)
@@ -199,7 +209,8 @@ class DecodeWorkload:
             self.call(m, s)
 
     def config(self):
-        form = " W8A8" if self.w8 else (" zero-point INT4" if self.zpf else "")
+        form = " W8A8" if self.w8 else (" zero-point INT4" if self.zpf else
+                                        (" group-wise INT4 (128)" if self.grp else ""))
         return {"workload": f"decode single linear{form} K={self.K} N={self.N} "
                             f"M in {list(self.MS)}",
                 "K": self.K, "N": self.N, "M": list(self.MS),
@@ -207,7 +218,8 @@ class DecodeWorkload:
                       f"({self.pool_bytes / 1e6:.0f} MB) rotate across launches",
                 "weights": "N(0,0.02) quantized" + ("" if self.w8 else "+packed") + " once before timing",
                 "activations": "N(0,1), 8 input channels x20",
-                "call": ("w8a8_linear" if self.w8 else "w4z_linear" if self.zpf else "w4a8_linear")
+                "call": ("w8a8_linear" if self.w8 else "w4z_linear" if self.zpf else
+                         "w4g_linear" if self.grp else "w4a8_linear")
                         + " with W4A8_STATIC_WEIGHTS"}
 
 
@@ -363,6 +375,8 @@ def time_kernel_only(torch, nat, wl):
         nbytes = wl.N * ldp + 4 * wl.N + m * xq.shape[1] + 4 * m + 4 * m * wl.N
         if getattr(wl, "zpf", False):
             nbytes += 4 * wl.N  # the zero points
+        if getattr(wl, "grp", False):
+            nbytes += 8 * wl.sw[0].numel() - 4 * wl.N  # per-group scales and zero points
         out[m] = (ms, nbytes, kernel)
     return out
 
@@ -515,11 +529,11 @@ def run_prefill(args, torch, native, synth, device, props, dist, world, rank, re
         print(json.dumps(line), flush=True)
 
 
-def run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank, zp=False):
+def run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank, zp=False, grp=False):
     """The decode workload on the W8A8 path (or, zp=True, the zero-point INT4
     path): the step (w8a8_linear / w4z_linear at M = 1, 4, 16, activation pass
     included) and the product call alone per M."""
-    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size, w8=not zp, zp=zp)
+    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size, w8=not (zp or grp), zp=zp, grp=grp)
     clocks = ClockSampler(device.index or 0)
     clocks.start()
     time.sleep(0.3)
@@ -537,15 +551,15 @@ def run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8xu4(zp)->s32" if zp else "s8xs8->s32",
+            "dtype": "s8xu4(zp)->s32" if zp else ("s8xu4(group zp)->f32" if grp else "s8xs8->s32"),
             "data": "synthetic", "config": wl.config(),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                         "traffic": None if zp else W8_DECODE_TRAFFIC_PER_LAUNCH,
+                         "traffic": None if (zp or grp) else W8_DECODE_TRAFFIC_PER_LAUNCH,
                          "traffic_note": "dram bytes read+written per k_linear8_decode launch, mean over M = 1, "
                                          "4, 16; ncu capture in profiles/k_linear8_decode_k4096_n4096.md",
                          "kernel": ("w4z_linear_q (row sums, product, zero-point epilogue)" if zp else
-                                    "k_linear8_decode") + " over M in " + str(list(kern)) +
+                                    "k_linear_g" if grp else "k_linear8_decode") + " over M in " + str(list(kern)) +
                                    " (back to back over rotating weights, static-weights promise)",
                          "per_m": {str(m): {"kernel": v[2], "us": round(v[0] * 1e3, 3), "bytes": v[1],
                                             "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
@@ -747,7 +761,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU work for the oracle baseline")
     ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep", "gemma-stack",
-                                           "decode-w8a8", "prefill-w8a8", "decode-zp"],
+                                           "decode-w8a8", "prefill-w8a8", "decode-zp", "decode-grp"],
                     default="decode",
                     help="decode (the headline line), prefill (M=2048 K=4096 N=11008), a per-shape "
                          "sweep of the other workloads, the 182-linear Gemma3-1B-shaped stack, or the "
@@ -790,9 +804,9 @@ def main():
         run_prefill(args, torch, native, synth, device, props, dist, world, rank,
                     relu=args.workload == "prefill-relu", w8=args.workload == "prefill-w8a8")
         return
-    if args.workload in ("decode-w8a8", "decode-zp"):
+    if args.workload in ("decode-w8a8", "decode-zp", "decode-grp"):
         run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank,
-                        zp=args.workload == "decode-zp")
+                        zp=args.workload == "decode-zp", grp=args.workload == "decode-grp")
         return
     if args.workload == "sweep":
         run_sweep(torch, native, synth, device, props)
