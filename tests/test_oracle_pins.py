@@ -620,3 +620,22 @@ def test_w4g_error_below_per_channel_zero_point():
     wpz, saz, zpz = oracle.w4z_quantize_pack(w)
     yz = oracle.linear_z(x, wpz, saz, zpz, 1024)
     assert np.abs(yg - exact).mean() < np.abs(yz - exact).mean()
+
+
+def test_zero_point_storage_identity():
+    """The algebra the zero-point kernels rely on, on the oracle alone: storing
+    each code as the signed nibble q - 8 and multiplying with the symmetric
+    INT4 product gives acc' = sum xq (q - 8); adding -(zp - 8) * sum xq gives
+    sum xq (q - zp), the zero-point product, exactly."""
+    rng = synth.rng_for(60, 0)
+    k, n, m = 333, 24, 7
+    w = rng.normal(0.0, 0.02, size=(k, n)).astype(np.float32)
+    w[:, 3] = np.abs(w[:, 3]) + 1.0  # a negative zero point
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    q = _unpack_unsigned(wp, k)
+    stored = oracle.w4_pack((q - 8).astype(np.int8))  # signed nibbles q - 8, pad 0
+    xq = rng.integers(-127, 128, size=(m, k)).astype(np.int8)
+    acc_prime = oracle.gemm_s32(xq, k, stored).astype(np.int64)
+    rowsum = xq.astype(np.int64).sum(axis=1)
+    acc = acc_prime - (zp.astype(np.int64)[None, :] - 8) * rowsum[:, None]
+    assert np.array_equal(acc, oracle.gemm_z_s32(xq, k, wp, zp).astype(np.int64))
