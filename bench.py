@@ -1,27 +1,37 @@
 #!/usr/bin/env python
 """Benchmark of the W4A8 per-channel linear layer on B200.
 
-Default workload: the decode single linear, K = N = 4096, activation rows
-M in {1, 4, 16}. One step = one pass of the run-time hot path over one batch:
-for each M, dynamic INT8 quantization of X[M][4096] and the W4A8 product with
-dequantization (w4a8_linear: two kernels). The weights are quantized and
-packed once, offline, before timing (their quantize+pack pass is timed on its
-own and reported under "stages").
+Default run: both halves of the metric on one JSON line.
+  * decode (the line's value): the decode single linear, K = N = 4096,
+    activation rows M in {1, 4, 16}. One step = one pass of the run-time hot
+    path over one batch: for each M, w4a8_linear (dynamic INT8 quantization of
+    X[M][4096], the W4A8 product, dequantization). HBM GB/s of algorithmic
+    bytes (packed weights + weight scales + float32 X + float32 Y per linear)
+    per second of device time. Weight buffers rotate through a pool of
+    distinct copies several times larger than L2, so every launch streams its
+    weights from HBM.
+  * prefill (the "prefill" sub-record): M = 2048, K = 4096, N = 11008,
+    float32 out; one step = one w4a8_linear (activation pass + tensor-core
+    GEMM + epilogue); TOPS = 2 M N K per second, and the GEMM kernel alone
+    against the dense INT8 tensor peak.
+The weights are quantized and packed once, offline, before timing (their
+quantize+pack pass is timed on its own and reported under "stages").
 
-Metric: HBM GB/s of algorithmic bytes (packed weights + weight scales +
-float32 X + float32 Y per linear) per second of device time. Weight buffers
-rotate through a pool of distinct copies several times larger than L2, so
-every launch streams its weights from HBM.
+Timing: CUDA graphs of the timed steps are built and replayed untimed first
+(warm-up), then the same graphs run the --steps-long region `repeats` times
+back to back, each bracketed by CUDA events on the launching stream; the
+reported time is the median region. Multi-GPU (torchrun): every rank runs the
+same independent workload (weak scaling, no collective on the data path);
+time is the max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill]
-
-Multi-GPU (torchrun): every rank runs the same independent workload (weak
-scaling, no collective on the data path); time is the max over ranks.
+                    [--workload decode|prefill|...]
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
+import hashlib
 import json
 import os
 import statistics
@@ -36,20 +46,46 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "W4A8 linear: TOPS (prefill) and HBM GB/s (decode) vs B200 roofline"
-# DRAM bytes (read + write) per launch of the decode product kernels at K = N = 4096, by kernel, from
-# the ncu captures summarized in profiles/ (k_decode_ring at M = 1; k_linear_decode: mean of its M = 4 and
-# M = 16 launches); recapture when a kernel changes.
-DECODE_TRAFFIC_PER_LAUNCH = {"k_decode_ring": 8433920, "k_linear_decode": 8460480}
-DECODE_TRAFFIC_NOTE = {
-    "k_decode_ring": "profiles/k_decode_ring_m1_k4096_n4096.md (M=1)",
-    "k_linear_decode": "profiles/launches_decode_bench_k4096_n4096.md (mean of M=4 and M=16)",
-}
-# The same for k_linear8_decode (W8A8 decode), mean over M = 1, 4, 16 (profiles/k_linear8_decode_k4096_n4096.md).
-W8_DECODE_TRAFFIC_PER_LAUNCH = 16834091
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernels, from ncu captures of this file's own workloads, stored
+# with a hash of the kernel sources they were taken on: a figure whose hash no
+# longer matches the sources is reported as null (stale).
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+KERNEL_SOURCES = (os.path.join(ROOT, "w4a8_quantized_gemm_channel_b200", "csrc"), os.path.join(ROOT, "include"))
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 INT8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
 GRAPH_STEPS = 16
+MIN_TIMED_S = 0.5      # repeat the timed region until this much device time is covered
+MAX_REPEATS = 2000
+
+
+def source_hash() -> str:
+    """sha256 over the kernel sources (csrc/*.cu, *.cuh and include/*.h)."""
+    h = hashlib.sha256()
+    for d in KERNEL_SOURCES:
+        for name in sorted(os.listdir(d)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                h.update(name.encode())
+                with open(os.path.join(d, name), "rb") as f:
+                    h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_for(kernel: str, workload: str):
+    """(bytes per launch, note) from the committed ncu figures, or (None, why)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None, "no ncu traffic figures committed"
+    e = d.get("kernels", {}).get(f"{kernel}@{workload}")
+    if e is None:
+        return None, f"no ncu capture of {kernel} on this workload"
+    if d.get("source_sha256") != source_hash():
+        return None, f"stale: the kernel sources changed since the ncu capture of {kernel}"
+    return e["dram_bytes_per_launch"], (f"dram__bytes_read.sum + dram__bytes_write.sum per {kernel} launch, "
+                                        f"{e.get('launches', '?')} captured launches ({e.get('case', workload)})")
 
 
 def measured_peaks():
@@ -261,7 +297,11 @@ class PrefillWorkload:
         return 2 * self.M * self.N * self.K
 
     def launches_per_step(self):
-        return 2
+        """Kernels one step enqueues, as the library reports them."""
+        self.step()
+        n = self.nat.last_launch_count()
+        self.torch.cuda.synchronize()
+        return n
 
     def step(self):
         s = self.slot
@@ -289,8 +329,8 @@ def max_over_ranks(torch, dist, value: float, device) -> float:
 
 
 def build_graphs(torch, wl, nsteps):
-    """CUDA graphs of GRAPH_STEPS steps (and one for the remainder)."""
-    graphs = []
+    """CUDA graphs that run exactly nsteps steps: `full` replays of one
+    GRAPH_STEPS-step graph, then one graph of the remainder."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
@@ -299,10 +339,12 @@ def build_graphs(torch, wl, nsteps):
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     full, rem = divmod(nsteps, GRAPH_STEPS)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for _ in range(GRAPH_STEPS):
-            wl.step()
+    g = None
+    if full:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(GRAPH_STEPS):
+                wl.step()
     gr = None
     if rem:
         gr = torch.cuda.CUDAGraph()
@@ -312,85 +354,55 @@ def build_graphs(torch, wl, nsteps):
     return g, full, gr
 
 
-def time_steps(torch, wl, steps, warmup, dist=None):
+def timed_repeats(torch, enqueue, dist=None, device=None, min_repeats=5):
+    """Median device time (ms) of one `enqueue()` (already warmed) over
+    back-to-back repeats, each bracketed by CUDA events on the current stream;
+    repeats run until MIN_TIMED_S of device time is covered (at least
+    min_repeats, at most MAX_REPEATS; the same count on every rank). Returns
+    (median ms, repeats)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    enqueue()
+    b.record()
+    torch.cuda.synchronize()
+    one = max(a.elapsed_time(b), 1e-3)
+    reps = int(min(MAX_REPEATS, max(min_repeats, -(-MIN_TIMED_S * 1e3 // one))))
+    reps = int(max_over_ranks(torch, dist, float(reps), device))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs[0].record()
+    for i in range(reps):
+        enqueue()
+        evs[i + 1].record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return statistics.median(evs[i].elapsed_time(evs[i + 1]) for i in range(reps)), reps
+
+
+def time_steps(torch, wl, steps, warmup, dist=None, device=None):
+    """Median device time (ms) of a region of exactly `steps` steps, and the
+    repeat count. The timed graphs themselves run the warm-up (at least
+    `warmup` steps, and every graph at least once), so no graph is replayed
+    for the first time inside a timed region."""
     g, full, gr = build_graphs(torch, wl, steps)
-    wg, wfull, wgr = build_graphs(torch, wl, warmup) if warmup else (None, 0, None)
-    for _ in range(wfull):
-        wg.replay()
-    if wgr is not None:
-        wgr.replay()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(full):
-        g.replay()
-    if gr is not None:
-        gr.replay()
-    stop.record()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    ms = start.elapsed_time(stop)
-    return ms
 
-
-def time_kernel_only(torch, nat, wl):
-    """Average device time per decode-kernel launch (w4a8_linear_q, INT8
-    activations already quantized) in a back-to-back graph over the rotating
-    weight pool, per M; returns {m: (ms_per_launch, algorithmic_bytes,
-    kernel_name)}."""
-    out = {}
-    ldp = wl.weight_ld()
-    for m in wl.MS:
-        xq, sx = nat.a8_quantize_rows(wl.x[m])
-        reps = wl.pool
-
-        def run():
-            for i in range(reps):
-                wl.linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], y=wl.y[m], static_weights=True)
-        wl.linear_q(xq, sx, wl.K, wl.wp[0], wl.sw[0], y=wl.y[m], static_weights=True)
-        kernel = nat.last_kernel()
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            run()
-        torch.cuda.current_stream().wait_stream(s)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            run()
-        for _ in range(3):
+    def region():
+        for _ in range(full):
             g.replay()
-        torch.cuda.synchronize()
-        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_rep = 20
-        start.record()
-        for _ in range(n_rep):
-            g.replay()
-        stop.record()
-        torch.cuda.synchronize()
-        ms = start.elapsed_time(stop) / (n_rep * reps)
-        nbytes = wl.N * ldp + 4 * wl.N + m * xq.shape[1] + 4 * m + 4 * m * wl.N
-        if getattr(wl, "zpf", False):
-            nbytes += 4 * wl.N  # the zero points
-        if getattr(wl, "grp", False):
-            nbytes += 8 * wl.sw[0].numel() - 4 * wl.N  # per-group scales and zero points
-        out[m] = (ms, nbytes, kernel)
-    return out
+        if gr is not None:
+            gr.replay()
+    for _ in range(max(1, -(-warmup // steps))):
+        region()
+    torch.cuda.synchronize()
+    return timed_repeats(torch, region, dist, device)
 
 
-def time_gemm_only(torch, nat, wl, reps=20):
-    """Average device time per tensor-core GEMM launch (w4a8_linear_q on INT8
-    activations) over the rotating buffer sets."""
-    m = wl.M
-    xqs = [nat.a8_quantize_rows(x) for x in wl.xs]
-    lin_q = nat.w8a8_linear_q if wl.w8 else nat.w4a8_linear_q
-    def run():
-        for i in range(wl.pool):
-            xq, sx = xqs[i]
-            lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
+def _graph_of(torch, run):
+    """Capture run() (after one eager warm-up on a side stream) and replay it
+    three times untimed."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
@@ -402,13 +414,50 @@ def time_gemm_only(torch, nat, wl, reps=20):
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(reps):
-        g.replay()
-    stop.record()
-    torch.cuda.synchronize()
-    return start.elapsed_time(stop) / (reps * wl.pool)
+    return g
+
+
+def time_kernel_only(torch, nat, wl):
+    """Device time per decode-kernel launch (w4a8_linear_q, INT8 activations
+    already quantized) in a back-to-back graph over the rotating weight pool,
+    per M (median over repeats of the graph); returns {m: (ms_per_launch,
+    algorithmic_bytes, kernel_name)}."""
+    out = {}
+    ldp = wl.weight_ld()
+    for m in wl.MS:
+        xq, sx = nat.a8_quantize_rows(wl.x[m])
+        reps = wl.pool
+
+        def run():
+            for i in range(reps):
+                wl.linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], y=wl.y[m], static_weights=True)
+        wl.linear_q(xq, sx, wl.K, wl.wp[0], wl.sw[0], y=wl.y[m], static_weights=True)
+        kernel = nat.last_kernel()
+        g = _graph_of(torch, run)
+        ms, _ = timed_repeats(torch, g.replay, min_repeats=20)
+        ms /= reps
+        nbytes = wl.N * ldp + 4 * wl.N + m * xq.shape[1] + 4 * m + 4 * m * wl.N
+        if getattr(wl, "zpf", False):
+            nbytes += 4 * wl.N  # the zero points
+        if getattr(wl, "grp", False):
+            nbytes += 8 * wl.sw[0].numel() - 4 * wl.N  # per-group scales and zero points
+        out[m] = (ms, nbytes, kernel)
+    return out
+
+
+def time_gemm_only(torch, nat, wl):
+    """Device time per tensor-core GEMM launch (w4a8_linear_q on INT8
+    activations) over the rotating buffer sets (median over repeats)."""
+    xqs = [nat.a8_quantize_rows(x) for x in wl.xs]
+    lin_q = nat.w8a8_linear_q if wl.w8 else nat.w4a8_linear_q
+
+    def run():
+        for i in range(wl.pool):
+            xq, sx = xqs[i]
+            lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
+    g = _graph_of(torch, run)
+    ms, _ = timed_repeats(torch, g.replay, min_repeats=20)
+    return ms / wl.pool
 
 
 def time_quantize_pack(torch, nat, wl):
@@ -454,58 +503,132 @@ def time_e2e(torch, nat, wl, steps):
     return start.elapsed_time(stop), h2d, d2h
 
 
+def time_e2e_prefill(torch, nat, wl, steps):
+    """The prefill step through w4a8_linear with host buffers: X copied in
+    from pinned memory and Y read back every step."""
+    xh = torch.from_numpy(wl.x_host[wl.M]).pin_memory()
+    yh = torch.empty((wl.M, wl.N), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(wl.xs[0])
+
+    def one(slot):
+        s = slot % wl.pool
+        xd.copy_(xh, non_blocking=True)
+        nat.w4a8_linear(xd, wl.wp[s], wl.sw[s], relu=wl.relu, y=wl.ys[s], workspace=wl.ws[wl.M])
+        yh.copy_(wl.ys[s], non_blocking=True)
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        one(i)
+    stop.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(stop), xh.numel() * 4, yh.numel() * 4
+
+
 # ------------------------------------------------------- the CPU oracle ---
 
-def oracle_decode_rate(budget_s: float, min_steps: int = 1):
-    """The oracle as it stands, on a bounded sample of the decode workload:
-    all three M values against a sample of output channels (full K)."""
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_columns(pool, oracle, xq, sx, wp, sw, k, c0, c1, per):
+    """oracle.linear_q on output channels [c0, c1) in tasks of `per` channels
+    spread over the thread pool (the oracle's C calls release the GIL)."""
+    jobs = [pool.submit(oracle.linear_q, xq, sx, wp[a:min(a + per, c1)], sw[a:min(a + per, c1)], k)
+            for a in range(c0, c1, per)]
+    return [j.result() for j in jobs]
+
+
+def oracle_decode_steps(budget_s: float, threads: int, min_steps: int = 1, max_steps: int | None = None):
+    """The oracle as it stands, timed on the decode workload at full size
+    (K = N = 4096, M = 1, 4, 16; per M the activation pass, then the product
+    and dequantization over all output channels split across `threads`
+    threads) until `budget_s` seconds are spent. Returns (GB/s of the decode
+    line's algorithmic bytes, seconds, steps)."""
     import oracle
     from w4a8_quantized_gemm_channel_b200 import synth
     k, n = synth.DECODE_K, synth.DECODE_N
-    w = synth.decode_case(1).w
+    wp, sw = oracle.w4_quantize_pack(synth.decode_case(1).w)   # offline step, not timed
     xs = {m: synth.decode_case(m).x for m in synth.DECODE_MS}
-    wp, sw = oracle.w4_quantize_pack(w)
     ldp = wp.shape[1]
-    cols = 64
-    done_bytes, t_used, chunks = 0, 0.0, 0
+    step_bytes = sum(n * ldp + 4 * n + 4 * m * k + 4 * m * n for m in xs)
+    per = max(8, n // (4 * threads))
+    steps = 0
+    with concurrent.futures.ThreadPoolExecutor(threads) as pool:
+        t0 = time.perf_counter()
+        while (time.perf_counter() - t0 < budget_s or steps < min_steps) and (max_steps is None or steps < max_steps):
+            for m, x in xs.items():
+                xq, sx = oracle.a8_quantize_rows(x)
+                _oracle_columns(pool, oracle, xq, sx, wp, sw, k, 0, n, per)
+            steps += 1
+        t = time.perf_counter() - t0
+    return steps * step_bytes / t / 1e9, t, steps
+
+
+def oracle_prefill_rate(budget_s: float, threads: int, case):
+    """The oracle on the prefill workload (M = 2048, K = 4096, N = 11008):
+    the activation pass over all of X, then the product on as many output
+    channels as `budget_s` seconds allow (full M and K, split across
+    `threads` threads). The full-layer time is extrapolated from that sample:
+    t = t_activation + t_sample * N / channels_done. Returns (TOPS, detail)."""
+    import oracle
+    x, w = case.x, case.w
+    m, k = x.shape
+    n = w.shape[1]
+    wp, sw = oracle.w4_quantize_pack(w)   # offline step, not timed
     t0 = time.perf_counter()
-    while (time.perf_counter() - t0 < budget_s) or chunks < min_steps:
-        c0 = (chunks * cols) % n
-        wps, sws = wp[c0:c0 + cols], sw[c0:c0 + cols]
-        for m, x in xs.items():
-            oracle.linear(x, wps, sws, k)
-            done_bytes += cols * ldp + 4 * cols + 4 * m * k + 4 * m * cols
-        chunks += 1
-    t_used = time.perf_counter() - t0
-    return done_bytes / t_used / 1e9, t_used, chunks, cols
+    xq, sx = oracle.a8_quantize_rows(x)
+    t_q = time.perf_counter() - t0
+    per, done, t_p = 4, 0, 0.0
+    with concurrent.futures.ThreadPoolExecutor(threads) as pool:
+        while done < n and (t_p < budget_s or done == 0):
+            c1 = min(n, done + per * threads)
+            t1 = time.perf_counter()
+            _oracle_columns(pool, oracle, xq, sx, wp, sw, k, done, c1, per)
+            t_p += time.perf_counter() - t1
+            done = c1
+    t_full = t_q + t_p * n / done
+    return 2.0 * m * n * k / t_full / 1e12, {"channels": done, "t_act_s": round(t_q, 3), "t_sample_s": round(t_p, 3)}
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle on the decode line's workload, on the
+    host cores, W untimed and K timed steps (each a full decode step, or a
+    bounded sample of one if the budget is too small for full steps)."""
     if rank != 0:
         return
-    budget = args.cpu_budget
-    gbs, t, chunks, cols = oracle_decode_rate(budget)
-    sample = (f"{chunks} samples of {cols} output channels x full K=4096 at M=1,4,16 "
-              f"({t:.1f} s single-threaded)")
+    threads = cpu_threads()
+    oracle_decode_steps(0.0, threads, min_steps=max(1, min(args.warmup, 3)), max_steps=max(1, min(args.warmup, 3)))
+    gbs, t, steps = oracle_decode_steps(args.cpu_budget, threads, min_steps=args.steps, max_steps=args.steps)
+    sample = f"{steps} full decode steps (M = 1, 4, 16; K = N = 4096) on {threads} threads, {t:.2f} s"
     line = {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "impl": "reference",
-            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
+            "ms_per_step": round(t * 1e3 / steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "decode single linear K=4096 N=4096 M in [1, 4, 16]",
-                       "note": "CPU oracle (plain C, one thread) on a bounded sample"},
-            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                       "note": "CPU oracle (plain C, one call per output-channel chunk, thread pool)"},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False):
+def prefill_record(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False,
+                   cpu=None):
+    """Time the prefill workload: the step (w4a8_linear, activation pass
+    included), the tensor-core GEMM alone, and the step through host buffers.
+    Returns the record (value in TOPS, with roofline, clocks and launches)."""
     wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu, w8=w8)
     clocks = ClockSampler(device.index or 0)
     clocks.start()
     time.sleep(0.3)
-    ms = time_steps(torch, wl, args.steps, args.warmup, dist)
+    ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device)
     ck = clocks.stop()
     ms = max_over_ranks(torch, dist, ms, device)
     tops = world * args.steps * wl.ops_per_step() / (ms * 1e-3) / 1e12
@@ -513,58 +636,114 @@ def run_prefill(args, torch, native, synth, device, props, dist, world, rank, re
     peaks, kind = measured_peaks()
     peak = INT8_OVER_BF16 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
     achieved = wl.ops_per_step() / (g_ms * 1e-3) / 1e12
-    line = {"metric": METRIC, "value": round(tops, 2), "unit": "TOPS", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8xs8->s32" if w8 else "s8xs4->s32",
-            "data": "synthetic", "config": wl.config(),
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
-                         "unit": "TOPS", "frac": round(achieved / peak, 4),
-                         "peak_source": f"{kind} bf16_tflops x {INT8_OVER_BF16:g} (nominal int8/bf16)",
-                         "traffic": None, "kernel": "k_gemm_tc (" + ("w8a8" if w8 else "w4a8")
-                                                    + "_linear_q, rotating buffers)",
-                         "us": round(g_ms * 1e3, 2)},
-            "gpu_launches": args.steps * wl.launches_per_step(), "clocks": ck}
+    traffic, tnote = traffic_for("k_gemm_tc", "prefill" + ("-w8a8" if w8 else "") + ("-relu" if relu else ""))
+    e2e_steps = min(args.steps, 10)
+    e_ms, h2d, d2h = time_e2e_prefill(torch, native, wl, e2e_steps) if not w8 else (None, 0, 0)
+    rec = {"value": round(tops, 2), "unit": "TOPS", "steps": args.steps, "repeats": repeats,
+           "ms_per_step": round(ms / args.steps, 6), "dtype": "s8xs8->s32" if w8 else "s8xs4->s32",
+           "config": wl.config(),
+           "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                        "unit": "TOPS", "frac": round(achieved / peak, 4),
+                        "peak_source": f"{kind} bf16_tflops (burst) x {INT8_OVER_BF16:g}, the nominal dense "
+                                       "int8/bf16 ratio (4.5 / 2.25 PFLOP/s)",
+                        "traffic": traffic, "traffic_note": tnote,
+                        "kernel": "k_gemm_tc (" + ("w8a8" if w8 else "w4a8") + "_linear_q back to back over "
+                                  "rotating buffers)", "us": round(g_ms * 1e3, 2)},
+           "gpu_launches": args.steps * wl.launches_per_step(), "clocks": ck}
+    if e_ms is not None:
+        rec["e2e"] = {"value": round(world * e2e_steps * wl.ops_per_step() / (e_ms * 1e-3) / 1e12, 2),
+                      "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+    if cpu is not None:
+        rec["cpu_baseline"] = cpu
+    del wl
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False, cpu=None):
+    rec = prefill_record(args, torch, native, synth, device, props, dist, world, rank, relu=relu, w8=w8, cpu=cpu)
+    line = {"metric": METRIC, "value": rec.pop("value"), "unit": rec.pop("unit"), "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rec.pop("dtype"),
+            "data": "synthetic", **rec}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank, zp=False, grp=False):
-    """The decode workload on the W8A8 path (or, zp=True, the zero-point INT4
-    path): the step (w8a8_linear / w4z_linear at M = 1, 4, 16, activation pass
-    included) and the product call alone per M."""
-    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size, w8=not (zp or grp), zp=zp, grp=grp)
+def decode_record(args, torch, native, synth, device, props, dist, world, form="w4"):
+    """Time the decode workload in one weight form ("w4": W4A8; "w8": W8A8;
+    "zp": zero-point INT4; "grp": group-wise INT4): the step (the form's
+    linear call at M = 1, 4, 16, activation quantization included), the
+    product call alone per M, the step through host buffers (W4A8) and the
+    offline weight pass (W4A8). Returns the line's fields."""
+    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size, w8=form == "w8", zp=form == "zp",
+                        grp=form == "grp")
     clocks = ClockSampler(device.index or 0)
     clocks.start()
     time.sleep(0.3)
-    ms = time_steps(torch, wl, args.steps, args.warmup, dist)
+    ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device)
     ck = clocks.stop()
     ms = max_over_ranks(torch, dist, ms, device)
     bytes_step = wl.bytes_per_step()
     value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9
+
     kern = time_kernel_only(torch, native, wl)
-    k_ms = sum(v[0] for v in kern.values())
-    k_bytes = sum(v[1] for v in kern.values())
+    # the dominant product kernel: the one with the most device time over the step's M
+    by_kernel = {}
+    for m, (_, _, name) in kern.items():
+        by_kernel.setdefault(name, []).append(m)
+    dom = max(by_kernel, key=lambda name: sum(kern[m][0] for m in by_kernel[name]))
+    dom_ms = by_kernel[dom]
+    k_ms = sum(kern[m][0] for m in dom_ms)
+    k_bytes = sum(kern[m][1] for m in dom_ms)
     peaks, peak_kind = measured_peaks()
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     achieved = k_bytes / (k_ms * 1e-3) / 1e9
-    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8xu4(zp)->s32" if zp else ("s8xu4(group zp)->f32" if grp else "s8xs8->s32"),
-            "data": "synthetic", "config": wl.config(),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_kind} hbm_gbs",
-                         "traffic": None if (zp or grp) else W8_DECODE_TRAFFIC_PER_LAUNCH,
-                         "traffic_note": "dram bytes read+written per k_linear8_decode launch, mean over M = 1, "
-                                         "4, 16; ncu capture in profiles/k_linear8_decode_k4096_n4096.md",
-                         "kernel": ("w4z_linear_q (row sums, product, zero-point epilogue)" if zp else
-                                    "k_linear_g" if grp else "k_linear8_decode") + " over M in " + str(list(kern)) +
-                                   " (back to back over rotating weights, static-weights promise)",
-                         "per_m": {str(m): {"kernel": v[2], "us": round(v[0] * 1e3, 3), "bytes": v[1],
-                                            "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
-                                   for m, v in kern.items()}},
-            "gpu_launches": args.steps * (4 if zp else 2) * len(wl.MS), "clocks": ck}
+    wname = {"w4": "decode", "w8": "decode-w8a8", "zp": "decode-zp", "grp": "decode-grp"}[form]
+    traffic, tnote = traffic_for(dom, wname)
+    call = {"w4": "w4a8_linear_q", "w8": "w8a8_linear_q", "zp": "w4z_linear_q", "grp": "w4g_linear_q"}[form]
+    rec = {
+        "value": round(value, 2), "unit": "GB/s", "steps": args.steps, "repeats": repeats,
+        "ms_per_step": round(ms / args.steps, 6),
+        "dtype": {"w4": "s8xs4->s32", "w8": "s8xs8->s32", "zp": "s8xu4(zp)->s32", "grp": "s8xu4(group zp)->f32"}[form],
+        "config": wl.config(),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic, "traffic_note": tnote,
+                     "kernel": f"{dom} over M in {dom_ms} ({call} back to back over rotating "
+                               "weights, static-weights promise); per_m lists every M's kernel",
+                     "per_m": {str(m): {"kernel": v[2], "us": round(v[0] * 1e3, 3), "bytes": v[1],
+                                        "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
+                               for m, v in kern.items()}},
+        "tops": round(world * args.steps * wl.ops_per_step() / (ms * 1e-3) / 1e12, 4),
+        "gpu_launches": args.steps * wl.launches_per_step(),
+        "gpu_launches_note": "kernels per timed region of `steps` steps (the region ran `repeats` times)",
+        "clocks": ck,
+    }
+    if form == "w4":
+        qp_ms, qp_bytes = time_quantize_pack(torch, native, wl)
+        rec["stages"] = {"quantize_pack": {"ms": round(qp_ms, 4), "bytes": qp_bytes,
+                                           "gbs": round(qp_bytes / (qp_ms * 1e-3) / 1e9, 1),
+                                           "frac_hbm": round(qp_bytes / (qp_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                                           "shape": f"K={wl.K} N={wl.N} fp32 -> packed"}}
+        e2e_steps = min(args.steps, 2000)
+        e2e_ms, h2d, d2h = time_e2e(torch, native, wl, e2e_steps)
+        rec["e2e"] = {"value": round(world * e2e_steps * bytes_step / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+    del wl
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank, zp=False, grp=False):
+    """The decode workload on the W8A8 path (or the zero-point / group-wise
+    INT4 paths): one JSON line."""
+    rec = decode_record(args, torch, native, synth, device, props, dist, world,
+                        form="zp" if zp else ("grp" if grp else "w8"))
+    line = {"metric": METRIC, "value": rec.pop("value"), "unit": rec.pop("unit"), "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rec.pop("dtype"),
+            "data": "synthetic", **rec}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -755,20 +934,28 @@ def run_gemma_stack(torch, native, synth, device, steps=20):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-budget", type=float, default=15.0,
-                    help="seconds of CPU work for the oracle baseline")
+    ap.add_argument("--cpu-budget", type=float, default=8.0,
+                    help="seconds of CPU work per oracle baseline (decode, prefill sample)")
     ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep", "gemma-stack",
                                            "decode-w8a8", "prefill-w8a8", "decode-zp", "decode-grp"],
                     default="decode",
-                    help="decode (the headline line), prefill (M=2048 K=4096 N=11008), a per-shape "
-                         "sweep of the other workloads, the 182-linear Gemma3-1B-shaped stack, or the "
-                         "decode / prefill workloads on the W8A8 path")
+                    help="decode (the default line: decode, with the prefill sub-record), prefill "
+                         "(M=2048 K=4096 N=11008) alone, a per-shape sweep of the other workloads, the "
+                         "182-linear Gemma3-1B-shaped stack, or the decode / prefill workloads on the "
+                         "W8A8, zero-point and group-wise paths")
+    ap.add_argument("--no-prefill", action="store_true", help="leave the prefill sub-record out of the default line")
+    ap.add_argument("--min-timed-s", type=float, default=MIN_TIMED_S,
+                    help="repeat each timed region until this much device time is covered (at least 5 "
+                         "repeats); a small value keeps profiler runs short")
     args = ap.parse_args()
+    globals()["MIN_TIMED_S"] = max(0.0, args.min_timed_s)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -789,20 +976,30 @@ def main():
         dist = dist_mod
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-
-    # the CPU baseline runs before any GPU work on rank 0 only, at N = 1
-    cpu = None
-    if rank == 0 and world == 1:
-        gbs, t, chunks, cols = oracle_decode_rate(args.cpu_budget)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"{chunks} samples of {cols} output channels x full K=4096 at M=1,4,16 "
-                         f"({t:.1f} s, single-threaded plain C)"}
-
     from w4a8_quantized_gemm_channel_b200 import native, synth
+
+    # the CPU baselines run before any GPU work, on rank 0 only, at N = 1
+    cpu = cpu_pf = None
+    threads = cpu_threads()
+    want_prefill = args.workload == "decode" and not args.no_prefill
+    if rank == 0 and world == 1:
+        if args.workload in ("decode", "prefill", "prefill-relu"):
+            if args.workload == "decode":
+                gbs, t, steps = oracle_decode_steps(args.cpu_budget, threads)
+                cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                       "sample": f"{steps} full decode steps (M = 1, 4, 16; K = N = 4096; every output "
+                                 f"channel) on {threads} threads, {t:.2f} s of plain-C oracle work"}
+            if want_prefill or args.workload != "decode":
+                tops, det = oracle_prefill_rate(args.cpu_budget, threads, synth.prefill_case())
+                cpu_pf = {"value": round(tops, 6), "unit": "TOPS", "cores": threads, "kind": "oracle",
+                          "sample": f"activation pass over all of X, then the product on {det['channels']} of "
+                                    f"{synth.PREFILL_N} output channels (full M and K) in {det['t_sample_s']} s "
+                                    f"on {threads} threads; the full-layer rate is extrapolated from that sample"}
+
     props = torch.cuda.get_device_properties(device)
     if args.workload in ("prefill", "prefill-relu", "prefill-w8a8"):
         run_prefill(args, torch, native, synth, device, props, dist, world, rank,
-                    relu=args.workload == "prefill-relu", w8=args.workload == "prefill-w8a8")
+                    relu=args.workload == "prefill-relu", w8=args.workload == "prefill-w8a8", cpu=cpu_pf)
         return
     if args.workload in ("decode-w8a8", "decode-zp", "decode-grp"):
         run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank,
@@ -814,61 +1011,17 @@ def main():
     if args.workload == "gemma-stack":
         run_gemma_stack(torch, native, synth, device)
         return
-    wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size)
 
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    ms = time_steps(torch, wl, args.steps, args.warmup, dist)
-    ck = clocks.stop()
-    ms = max_over_ranks(torch, dist, ms, device)
-    bytes_step = wl.bytes_per_step()
-    value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9
-
-    kern = time_kernel_only(torch, native, wl)
-    # the dominant product kernel: the one with the most device time over the step's M
-    by_kernel = {}
-    for m, (t_ms, nbytes, name) in kern.items():
-        by_kernel.setdefault(name, []).append(m)
-    dom = max(by_kernel, key=lambda name: sum(kern[m][0] for m in by_kernel[name]))
-    dom_ms = by_kernel[dom]
-    k_ms = sum(kern[m][0] for m in dom_ms)
-    k_bytes = sum(kern[m][1] for m in dom_ms)
-    peaks, peak_kind = measured_peaks()
-    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
-    achieved = k_bytes / (k_ms * 1e-3) / 1e9
-    qp_ms, qp_bytes = time_quantize_pack(torch, native, wl)
-    e2e_steps = min(args.steps, 2000)
-    e2e_ms, h2d, d2h = time_e2e(torch, native, wl, e2e_steps)
-    e2e_val = world * e2e_steps * bytes_step / (e2e_ms * 1e-3) / 1e9
-
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 6),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8xs4->s32",
-        "data": "synthetic", "config": wl.config(),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
-                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": DECODE_TRAFFIC_PER_LAUNCH.get(dom),
-                     "traffic_note": f"dram bytes read+written per {dom} launch, ncu capture in "
-                                     f"{DECODE_TRAFFIC_NOTE.get(dom, '(none)')}",
-                     "kernel": f"{dom} over M in {dom_ms} (w4a8_linear_q back-to-back over rotating "
-                               "weights, static-weights promise); per_m lists every M's kernel",
-                     "per_m": {str(m): {"kernel": v[2], "us": round(v[0] * 1e3, 3), "bytes": v[1],
-                                        "gbs": round(v[1] / (v[0] * 1e-3) / 1e9, 1)}
-                               for m, v in kern.items()}},
-        "stages": {"quantize_pack": {"ms": round(qp_ms, 4), "bytes": qp_bytes,
-                                     "gbs": round(qp_bytes / (qp_ms * 1e-3) / 1e9, 1),
-                                     "frac_hbm": round(qp_bytes / (qp_ms * 1e-3) / 1e9 / hbm_peak, 4),
-                                     "shape": f"K={wl.K} N={wl.N} fp32 -> packed"}},
-        "tops": round(world * args.steps * wl.ops_per_step() / (ms * 1e-3) / 1e12, 4),
-        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps * wl.launches_per_step(),
-        "clocks": ck,
-    }
+    rec = decode_record(args, torch, native, synth, device, props, dist, world, form="w4")
+    line = {"metric": METRIC, "value": rec.pop("value"), "unit": rec.pop("unit"), "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rec.pop("dtype"),
+            "data": "synthetic", **rec}
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if want_prefill:
+        line["prefill"] = prefill_record(args, torch, native, synth, device, props, dist, world, rank, cpu=cpu_pf)
+        line["gpu_launches"] += line["prefill"]["gpu_launches"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

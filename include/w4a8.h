@@ -188,6 +188,11 @@ W4A8_API w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx,
                                          const float *bias, unsigned flags,
                                          void *Y, int ldy, void *stream);
 
+/* The size in bytes of w4a8_linear_noalloc's scratch array as this library
+ * was built (W4A8_NOALLOC_SCRATCH_BYTES), for callers that do not compile
+ * against this header. */
+W4A8_API size_t w4a8_noalloc_scratch_bytes(void);
+
 /*
  * w4a8_linear_grouped - many independent few-row linears (steps 3-6 each) in
  * as few launches as possible: one persistent launch per 64 problems. Meant

@@ -336,7 +336,8 @@ def test_linear_q_full_code_range(nat, path):
 
 def test_tc_large_k_uses_sign_extension(nat):
     """K above the limit of the tensor-core kernel's 16*q byte trick
-    (16 * 128 * 127 * K must stay below 2^31) still gives exact results."""
+    (each term 16 q * xq is at most 128 * 127 in size, so 128 * 127 * K must
+    stay below 2^31) still gives exact results."""
     m, k, n = 20, 140000, 16
     x, w, _ = _case(m, k, n, seed=900)
     wp, sw = oracle.w4_quantize_pack(w)
@@ -514,3 +515,30 @@ def test_grouped_decode_many_problems_and_static_weights(nat):
     for (xd, wpd, swd, bd), y in zip(dp, ys):
         y1 = nat.w4a8_linear(xd, wpd, swd, bias=bd)
         assert np.array_equal(host(y).view(np.uint32), host(y1).view(np.uint32))
+
+
+@pytest.mark.parametrize("path", ["tc", "decode", "generic"])
+def test_extreme_scale_products(nat, path):
+    """Rows and weight columns whose scales are finite but whose product
+    sx * sw leaves the normal float32 range: row 0 has abs-max ~1e-28
+    (sx ~1.3e30) and meets a weight column of abs-max ~1e-9 (sw ~7e9), so
+    sx * sw overflows to inf and y = acc / inf is a signed zero; row 1 has
+    abs-max ~1e30 (sx ~1.3e-28) and meets a column of abs-max ~1e20
+    (sw ~7e-20), so sx * sw underflows to 0 and y = acc / 0 is infinite.
+    Every path must give the oracle's IEEE results there, and the 1e-6 bar
+    elsewhere."""
+    m, k, n = 40, 512, 48
+    x, w, _ = _case(m, k, n, seed=990)
+    x[0] *= 1e-28
+    x[1] *= 1e30
+    w[:, 0] *= 1e-9 / 0.02
+    w[:, 1] *= 1e20 / 0.02
+    wp, sw = oracle.w4_quantize_pack(w)
+    ref = oracle.linear(x, wp, sw, k)
+    got = host(nat.w4a8_linear(dev(x), dev(wp), dev(sw), path=path))
+    special = ~np.isfinite(ref) | (ref == 0)
+    assert special[0, 0] and special[1, 1]
+    signed = special & ~np.isnan(ref)          # a NaN's sign bit is not defined by IEEE division
+    assert np.array_equal(np.signbit(got[signed]), np.signbit(ref[signed]))
+    assert np.array_equal(got[special], ref[special], equal_nan=True)
+    assert_f32_close(np.where(special, 1.0, got), np.where(special, 1.0, ref))

@@ -81,7 +81,8 @@ constexpr int A_COLS = BK / 4;     // TMEM columns per A slot (4 INT8 per column
 //      exactly 16*q as INT8 (q in [-8, 7] gives 16q in [-128, 112]); the
 //      accumulator is then exactly 16*acc and the epilogue shifts it back.
 //      Two masks and one shift per 8 codes, plus the two byte permutes.
-//      Needs 16 * 128 * 127 * K < 2^31, i.e. K <= TC_X16_MAX_K.
+//      Each term 16 q * xq is at most 128 * 127 in size, so this needs
+//      128 * 127 * K < 2^31, i.e. K <= TC_X16_MAX_K.
 //  UNPACK_X16_PERM: as UNPACK_X16 without the byte permutes: the activations
 //      were stored with each group of 8 k reordered to k0 k2 k4 k6 k1 k3 k5 k7
 //      (see k_act_quant), which is the order the masks produce.
@@ -149,6 +150,10 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&v)[32], void *__restr
             const float q0 = __fmul_rn(f, r);
             const float e = __fmaf_rn(-q0, d, f);
             float y = __fmaf_rn(e, r, q0);
+            // The correction needs a normal 1/d and a finite f * r (|f| < 2^31):
+            // outside 2^-94 <= d <= 2^126 (extreme scales whose product is tiny,
+            // huge or overflows) take the IEEE division itself.
+            if (!(d >= 0x1p-94f && d <= 0x1p126f)) y = __fdiv_rn(f, d);
             if constexpr (BIAS) y = __fadd_rn(y, bn);
             if constexpr (RELU) y = y > 0.0f ? y : 0.0f;
             if constexpr (FMT == EPI_BF16) {

@@ -798,6 +798,8 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
                            static_cast<cudaStream_t>(stream));
 }
 
+size_t w4a8_noalloc_scratch_bytes(void) { return (size_t)W4A8_NOALLOC_SCRATCH_BYTES; }
+
 w4a8_status w8a8_linear(const float *X, int M, int K, int ldx, const int8_t *Wq, int ldw8,
                         const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
                         void *workspace, size_t workspace_bytes, void *stream) {

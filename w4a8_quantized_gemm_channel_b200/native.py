@@ -47,6 +47,7 @@ SIGNATURES = {
     "w4a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
     "w4a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
+    "w4a8_noalloc_scratch_bytes": (_S, []),
     "w8a8_ld": (_I, [_I]),
     "w8_quantize": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     "w8a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
@@ -226,7 +227,8 @@ def w4a8_linear_grouped(problems, relu: bool = False, out: str = "f32", stream=N
     return ys
 
 
-NOALLOC_SCRATCH_BYTES = 16 << 20
+# the library's own figure, so Python and C cannot drift apart
+NOALLOC_SCRATCH_BYTES = lib.w4a8_noalloc_scratch_bytes()
 
 
 def w4a8_linear_noalloc(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
