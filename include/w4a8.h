@@ -78,9 +78,14 @@ enum {
 /* Kernel selection. AUTO picks by shape; the others force one kernel (tests). */
 #define W4A8_PATH_AUTO     0x00u
 #define W4A8_PATH_GENERIC  0x10u /* CUDA-core kernel, any shape */
-#define W4A8_PATH_DECODE   0x20u /* weight-streaming kernel for few rows (M <= 16 per tile) */
+#define W4A8_PATH_DECODE   0x20u /* weight-streaming kernel for few rows (M <= 16 per tile), picked by shape */
 #define W4A8_PATH_TC       0x30u /* tcgen05 tensor-core GEMM (INT32 accumulators in TMEM) */
-#define W4A8_PATH_MASK     0x30u
+/* One kernel of the decode family, forced (W4A8_ERR_UNSUPPORTED where it
+ * cannot run the shape); w4a8_last_path reports them as W4A8_PATH_DECODE. */
+#define W4A8_PATH_DECODE_RING  0x40u /* k_decode_ring: persistent TMA ring, M <= 8, K <= 131072 */
+#define W4A8_PATH_DECODE_REGS  0x50u /* k_linear_decode: weights in registers, any M in tiles of 16 */
+#define W4A8_PATH_DECODE_SPLIT 0x60u /* k_decode_split: cluster K-split, M <= 16, K <= 8192 */
+#define W4A8_PATH_MASK     0x70u
 
 /* Largest K whose INT32 accumulator cannot overflow: 127 * 8 * K < 2^31. */
 #define W4A8_MAX_K 2097152
@@ -192,6 +197,47 @@ W4A8_API w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx,
  * was built (W4A8_NOALLOC_SCRATCH_BYTES), for callers that do not compile
  * against this header. */
 W4A8_API size_t w4a8_noalloc_scratch_bytes(void);
+
+/*
+ * Layer chaining - one Dense layer feeding the next (the guide's minimal model,
+ * section "Quantize a minimal functional model": each layer quantizes its own
+ * float32 input dynamically, step 3 of "How it works"). The activation step
+ * of a layer needs the abs-max of each of its input rows, which is a
+ * reduction over the previous layer's whole output row. w4a8_linear_chain
+ * lets the previous layer hand it over: with y_amax it also writes, for
+ * every output row m and every 16 consecutive output channels p,
+ *   y_amax[m][p] = max over n in [16 p, 16 p + 16) of |Y[m][n]|
+ * (of the stored float32 outputs, after bias and ReLU), so that the next
+ * layer's row abs-max is max_p y_amax[m][p] - exactly max_n |Y[m][n]| - and it
+ * can quantize its rows inside its product kernel without a pass over them.
+ * The pages have no API of their own for this; the results are those of
+ * w4a8_linear bit for bit.
+ */
+
+/* Parts per output row of y_amax for N output channels: ceil(N / 16); -1 if N < 1. */
+W4A8_API int w4a8_amax_parts(int N);
+
+/*
+ * w4a8_linear_chain - w4a8_linear with float32 output that takes and gives
+ * per-row abs-max parts.
+ *   X, Wp, sw, bias, Y, workspace: as for w4a8_linear; Y is float32.
+ *   x_amax  [M][x_parts] float32 or NULL: parts whose max over a row equals
+ *           max_k |X[m][k]| (such as the y_amax of the layer that wrote X);
+ *           NULL: the call reduces the rows itself. A wrong x_amax gives
+ *           wrong scales, not an error.
+ *   y_amax  [M][w4a8_amax_parts(N)] float32 out, or NULL.
+ *   flags   W4A8_RELU | W4A8_STATIC_WEIGHTS | one W4A8_PATH_*; any output
+ *           format other than W4A8_OUT_F32 is W4A8_ERR_INVALID_ARG.
+ * Launches: one on the generic and the cluster K-split decode kernels (the
+ * activation step runs inside the product kernel); otherwise the activation
+ * pass and the product, plus one pass over Y when y_amax is asked for.
+ */
+W4A8_API w4a8_status w4a8_linear_chain(const float *X, int M, int K, int ldx,
+                                       const float *x_amax, int x_parts,
+                                       const uint8_t *Wp, int ldp, const float *sw, int N,
+                                       const float *bias, unsigned flags,
+                                       float *Y, int ldy, float *y_amax,
+                                       void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * w4a8_linear_grouped - many independent few-row linears (steps 3-6 each) in
@@ -362,15 +408,15 @@ W4A8_API w4a8_status w4g_linear_q(const int8_t *Xq, int M, int K, int ldq, const
 W4A8_API unsigned w4a8_last_path(void);
 
 /* How many kernels the calling thread's last successful w4a8_linear /
- * w4a8_linear_q / w4a8_linear_noalloc call enqueued (1 or 2; 0 if none, or
- * if that call had M == 0). */
+ * w4a8_linear_q / w4a8_linear_noalloc / w4a8_linear_chain call enqueued
+ * (1 to 3; 0 if none, or if that call had M == 0). */
 W4A8_API unsigned w4a8_last_launch_count(void);
 
 /* Name of the product kernel that the calling thread's last successful
- * w4a8_linear / w4a8_linear_q / w4a8_linear_noalloc / w4a8_linear_grouped /
- * w8a8_linear / w8a8_linear_q
- * call enqueued ("k_decode_ring", "k_linear_decode", "k_gemm_tc",
- * "k_linear_generic", "k_decode_grouped", or for the W8A8 calls
+ * w4a8_linear / w4a8_linear_q / w4a8_linear_noalloc / w4a8_linear_chain /
+ * w4a8_linear_grouped / w8a8_linear / w8a8_linear_q
+ * call enqueued ("k_decode_split", "k_decode_ring", "k_linear_decode",
+ * "k_gemm_tc", "k_linear_generic", "k_decode_grouped", or for the W8A8 calls
  * "k_linear8_decode", "k_linear8_generic", "k_gemm_tc"), not counting the activation
  * pass; "" if none, or if that call had nothing to do. A static string that
  * the caller must not free. */

@@ -237,17 +237,20 @@ def test_decode_full_size(nat, m):
     assert np.array_equal(host(acc), oracle.linear(c.x, wp, sw, synth.DECODE_K, out="s32"))
 
 
-@pytest.mark.parametrize("m,k,groups_over_2sm,kernel", [
-    (1, 4096, -40, "k_decode_ring"), (2, 4096, -40, "k_decode_ring"), (3, 4096, -40, "k_linear_decode"),
-    (8, 4096, -290, "k_linear_decode"), (8, 4097, -290, "k_decode_ring"), (8, 4096, 0, "k_linear_decode"),
-    (8, 4096, 1, "k_decode_ring"), (16, 4096, -40, "k_linear_decode")])
-def test_decode_kernel_choice_and_bits(nat, m, k, groups_over_2sm, kernel):
-    """Few-row products with INT8 input on both sides of the rule that hands
-    short layers (at most two 16-channel groups per SM) with K <= 4096 and
-    M >= 3 to the register-path kernel: the kernel named, and the INT32
-    accumulators bit for bit, with and without the static-weights promise."""
+@pytest.mark.parametrize("m,k,blocks_over_2sm,kernel", [
+    (1, 4096, -5, "k_decode_split"), (16, 4096, -5, "k_decode_split"), (16, 4096, 0, "k_decode_split"),
+    (1, 4096, 1, "k_decode_ring"), (2, 4096, 1, "k_decode_ring"), (8, 4096, 1, "k_decode_ring"),
+    (12, 4096, 1, "k_linear_decode"), (1, 8193, -40, "k_decode_ring"), (12, 8193, -40, "k_linear_decode")])
+def test_decode_kernel_choice_and_bits(nat, m, k, blocks_over_2sm, kernel):
+    """Few-row products with INT8 input on both sides of the selection rule:
+    short layers (their K-split CTAs, 128 channels x one K slice each, fit two
+    per SM: at K = 4096, 8 slices, so 2 SMs / 8 blocks of 128 channels) take
+    the cluster K-split kernel; longer layers, and K beyond its 8 x 8 chunks,
+    the persistent ring for M <= 8 and the register kernel above. The kernel
+    named, and the INT32 accumulators bit for bit, with and without the
+    static-weights promise."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    n = 16 * (2 * sms + groups_over_2sm)
+    n = 128 * ((2 * sms) // 8 + blocks_over_2sm) if k == 4096 else 64 * (40 + blocks_over_2sm + 1)
     x, w, _ = _case(m, k, n, seed=1300 + m + k)
     wp, sw = oracle.w4_quantize_pack(w)
     ref = oracle.linear(x, wp, sw, k, out="s32")
@@ -399,18 +402,19 @@ def test_fused_decode_bit_exact(nat, m, k, pad):
 @pytest.mark.parametrize("m,k", [(1, 8192), (1, 8193), (2, 4096), (2, 4097), (4, 2048), (4, 2049),
                                  (1, 65536), (1, 65537), (2, 32768), (2, 32769), (4, 16384), (4, 16385),
                                  (8, 8192), (8, 8193)])
-def test_decode_at_kernel_boundaries(nat, m, k):
+@pytest.mark.parametrize("path", ["decode", "ring"])
+def test_decode_at_kernel_boundaries(nat, m, k, path):
     """Both sides of every K at which the few-row decode changes kernels: the
-    activation quantization still fits the product kernel's registers; one
-    weight stage and the INT8 rows still fit a block's shared memory. The
-    result must not depend on the side, with or without the static-weights
-    promise."""
+    K-split kernel's 8 x 8 chunks of 128 k (K = 8192); the ring kernel's
+    in-register activation quantization; one ring stage and the INT8 rows in
+    a block's shared memory. The result must not depend on the side, with or
+    without the static-weights promise."""
     n = 24
     x, w, _ = _case(m, k, n, seed=1200 + m)
     wp, sw = oracle.w4_quantize_pack(w)
     ref = oracle.linear(x, wp, sw, k, out="s32")
     for static in (False, True):
-        acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32", path="decode", static_weights=static)
+        acc = nat.w4a8_linear(dev(x), dev(wp), dev(sw), out="s32", path=path, static_weights=static)
         assert np.array_equal(host(acc), ref)
 
 
@@ -517,20 +521,21 @@ def test_grouped_decode_many_problems_and_static_weights(nat):
         assert np.array_equal(host(y).view(np.uint32), host(y1).view(np.uint32))
 
 
-@pytest.mark.parametrize("path", ["tc", "decode", "generic"])
+@pytest.mark.parametrize("path", ["tc", "decode", "generic", "split", "ring", "regs"])
 def test_extreme_scale_products(nat, path):
     """Rows and weight columns whose scales are finite but whose product
-    sx * sw leaves the normal float32 range: row 0 has abs-max ~1e-28
-    (sx ~1.3e30) and meets a weight column of abs-max ~1e-9 (sw ~7e9), so
+    sx * sw leaves the normal float32 range: row 0 has abs-max ~5e-32
+    (sx ~2.5e33) and meets a weight column of abs-max ~3e-9 (sw ~2.2e9), so
     sx * sw overflows to inf and y = acc / inf is a signed zero; row 1 has
-    abs-max ~1e30 (sx ~1.3e-28) and meets a column of abs-max ~1e20
-    (sw ~7e-20), so sx * sw underflows to 0 and y = acc / 0 is infinite.
-    Every path must give the oracle's IEEE results there, and the 1e-6 bar
-    elsewhere."""
-    m, k, n = 40, 512, 48
+    abs-max ~2.4e34 (sx ~5e-33) and meets a column of abs-max ~3.4e20
+    (sw ~2e-20), so sx * sw underflows to 0 and y = acc / 0 is infinite; row
+    1 against the ordinary columns gives sx * sw ~2^-100, below the range of
+    the reciprocal form. Every path must give the oracle's IEEE results there,
+    and the 1e-6 bar elsewhere."""
+    m, k, n = (8 if path in ("split", "ring") else 40), 512, 48
     x, w, _ = _case(m, k, n, seed=990)
-    x[0] *= 1e-28
-    x[1] *= 1e30
+    x[0] *= 1e-33
+    x[1] *= 1e33
     w[:, 0] *= 1e-9 / 0.02
     w[:, 1] *= 1e20 / 0.02
     wp, sw = oracle.w4_quantize_pack(w)

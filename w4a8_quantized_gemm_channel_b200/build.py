@@ -26,6 +26,9 @@ NVCC_FLAGS = [
     # exactly like the method's statement.
     "-prec-div=true", "-fmad=false",
     "--expt-relaxed-constexpr",
+    # compile the kernels of the one translation unit in parallel (ptxas runs
+    # per kernel; one thread per host core)
+    "--split-compile=0",
 ]
 
 

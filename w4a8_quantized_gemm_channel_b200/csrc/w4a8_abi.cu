@@ -15,6 +15,8 @@
 #include "zero_point.cuh"
 #include "group_wise.cuh"
 #include "decode_bulk.cuh"
+#include "decode_split.cuh"
+#include "chain.cuh"
 #include "gemm_tc.cuh"
 
 namespace w4a8 {
@@ -111,8 +113,13 @@ w4a8_status check_common(int M, int K, int N, const uint8_t *Wp, int ldp, const 
     const size_t esz = fmt == W4A8_OUT_BF16 ? 2 : 4;
     if ((reinterpret_cast<uintptr_t>(Y) & (esz - 1)) != 0) return W4A8_ERR_INVALID_ARG;
     if (flags & ~(W4A8_RELU | W4A8_OUT_MASK | W4A8_STATIC_WEIGHTS | W4A8_PATH_MASK)) return W4A8_ERR_INVALID_ARG;
+    if ((flags & W4A8_PATH_MASK) > W4A8_PATH_DECODE_SPLIT) return W4A8_ERR_INVALID_ARG;
     return W4A8_OK;
 }
+
+// The family (generic, decode, tensor core) of a path value: the forced
+// decode kernels belong to the decode family.
+inline unsigned path_family(unsigned path) { return path >= W4A8_PATH_DECODE_RING ? W4A8_PATH_DECODE : path; }
 
 // Kernel selection by shape. Few rows: the layer is a weight stream, so the
 // decode kernel; many rows: the tensor-core GEMM; tiny problems: generic.
@@ -227,8 +234,8 @@ int fq_j8(int K) {  // units per row and thread to cover the stages' k, rounded 
     return p;
 }
 bool fq_in_registers(int M, int K) { return fq_rows(M) * fq_j8(K) <= 4; }
-bool fq_eligible(int M, int K, int N, unsigned path) {
-    if (path != W4A8_PATH_DECODE || M > 4) return false;
+bool fq_eligible(int M, int K, int N) {
+    if (M > 4) return false;
     const RingPlan plan = ring_plan(M, K, N);
     return plan.ok && (fq_in_registers(M, K) || (long long)plan.grid * M * 16 <= N);
 }
@@ -266,6 +273,17 @@ w4a8_status launch_fq(const float *X, int M, int K, int ldx, const uint8_t *Wp, 
     return W4A8_OK;
 }
 
+// The cluster K-split kernel serves short layers: those whose CTAs (128
+// channels x one K slice each) fit two per SM in one wave, so that the whole
+// weight stream is requested before the dependency wait and nothing but the
+// slice's activations, the MMAs and one cluster reduction remain after it.
+// Long layers keep the persistent ring (or the register kernel), which stream
+// many waves of weights per block.
+bool split_preferred(int M, int K, int N) {
+    const dsplit::Plan pl = dsplit::plan(M, K, N);
+    return pl.ok && (long long)pl.nblk * pl.C <= 2LL * device_info().sm_count;
+}
+
 // On a short layer (at most two 16-channel groups per SM) whose packed rows
 // are one batch of k_linear_decode<1> (K <= 4096), that kernel beats the ring
 // from M = 3 rows on: each thread holds its whole share of the weights in
@@ -281,6 +299,55 @@ bool registers_beat_ring(int M, int K, int N) {
            groups <= 2LL * device_info().sm_count;
 }
 
+enum DecodeKernel { DK_NONE = 0, DK_SPLIT, DK_RING, DK_REGS };
+
+// The decode kernel for a path value of the decode family: the forced one if
+// it can run the shape (DK_NONE if not), else the rule by shape.
+DecodeKernel decode_kernel_for(unsigned path, int M, int K, int N) {
+    if (path == W4A8_PATH_DECODE_SPLIT) return dsplit::plan(M, K, N).ok ? DK_SPLIT : DK_NONE;
+    if (path == W4A8_PATH_DECODE_RING) return ring_plan(M, K, N).ok ? DK_RING : DK_NONE;
+    if (path == W4A8_PATH_DECODE_REGS) return DK_REGS;
+    if (split_preferred(M, K, N)) return DK_SPLIT;
+    if (ring_plan(M, K, N).ok && !registers_beat_ring(M, K, N)) return DK_RING;
+    return DK_REGS;
+}
+
+// One launch of the cluster K-split kernel. in: dsplit::IN_*; for IN_Q the
+// activations are (Xq, ldq, sx), otherwise (X, ldx) with x_amax/x_parts for
+// IN_F32_PARTS. y_amax: the chaining output, or null.
+cudaError_t launch_split(int in, const int8_t *Xq, int ldq, const float *sx, const float *X, int ldx,
+                         const float *x_amax, int x_parts, int M, int K, const uint8_t *Wp, int ldp,
+                         const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
+                         float *y_amax, bool early, cudaStream_t s) {
+    const dsplit::Plan pl = dsplit::plan(M, K, N);
+    if (!pl.ok) return cudaErrorInvalidValue;
+    dsplit::Params p = {};
+    p.Xq = Xq;
+    p.sx = sx;
+    p.ldq = ldq;
+    p.X = X;
+    p.ldx = ldx;
+    p.vec4 = X != nullptr && aligned16(X) && (ldx % 4 == 0);
+    p.x_amax = x_amax;
+    p.x_parts = x_parts;
+    p.M = M;
+    p.K = K;
+    p.Wp = Wp;
+    p.ldp = ldp;
+    p.sw = sw;
+    p.N = N;
+    p.bias = bias;
+    p.flags = flags;
+    p.Y = Y;
+    p.ldy = ldy;
+    p.y_amax = y_amax;
+    p.y_parts = (N + 15) / 16;
+    p.ch = pl.ch;
+    if (in == dsplit::IN_Q) return dsplit::launch<dsplit::IN_Q>(pl, p, early, s);
+    if (in == dsplit::IN_F32) return dsplit::launch<dsplit::IN_F32>(pl, p, early, s);
+    return dsplit::launch<dsplit::IN_F32_PARTS>(pl, p, early, s);
+}
+
 // act_perm: Xq uses the k-permuted layout (only the tensor-core path reads it).
 // after_act_pass: the launch directly follows this library's activation pass,
 // so the decode kernel may stream its weights before its dependency wait (as
@@ -292,30 +359,36 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
     const unsigned path = choose_path(M, K, N, flags);
-    if (act_perm && path != W4A8_PATH_TC) return W4A8_ERR_INVALID_ARG;
+    const unsigned fam = path_family(path);
+    if (act_perm && fam != W4A8_PATH_TC) return W4A8_ERR_INVALID_ARG;
+    const DecodeKernel dk = fam == W4A8_PATH_DECODE ? decode_kernel_for(path, M, K, N) : DK_NONE;
+    if (fam == W4A8_PATH_DECODE && dk == DK_NONE) return W4A8_ERR_UNSUPPORTED;
+    const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
     cudaError_t e = cudaSuccess;
     const char *kernel = "";
-    if (path == W4A8_PATH_GENERIC) {
+    if (fam == W4A8_PATH_GENERIC) {
         kernel = "k_linear_generic";
         dim3 grid((N + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
         e = launch_pdl(k_linear_generic, grid, dim3(128), 0, stream,
                        Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
-    } else if (path == W4A8_PATH_DECODE && ring_plan(M, K, N).ok && !registers_beat_ring(M, K, N)) {
+    } else if (dk == DK_SPLIT) {
+        kernel = "k_decode_split";
+        e = launch_split(dsplit::IN_Q, Xq, ldq, sx, nullptr, 0, nullptr, 0, M, K, Wp, ldp, sw, N, bias, flags, Y,
+                         ldy, nullptr, early, stream);
+    } else if (dk == DK_RING) {
         kernel = "k_decode_ring";
-        const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
         e = launch_ring_q(ring_plan(M, K, N), early, Xq, ldq, sx, M, K, Wp, ldp, sw, N, bias, flags, Y, ldy, stream);
-    } else if (path == W4A8_PATH_DECODE) {
+    } else if (dk == DK_REGS) {
         kernel = "k_linear_decode";
         const int tok = M <= 8 ? 8 : 16;
         const int tiles = (M + tok - 1) / tok;
         if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
         dim3 grid((N + 15) / 16, tiles);
-        const bool early = after_act_pass || (flags & W4A8_STATIC_WEIGHTS);
         auto kern = tok == 8 ? (early ? k_linear_decode<1, true> : k_linear_decode<1, false>)
                              : (early ? k_linear_decode<2, true> : k_linear_decode<2, false>);
         e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream,
                        Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
-    } else if (path == W4A8_PATH_TC) {
+    } else if (fam == W4A8_PATH_TC) {
         kernel = "k_gemm_tc";
         if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
         w4a8_status st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
@@ -325,7 +398,7 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
         return W4A8_ERR_INVALID_ARG;
     }
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
-    t_last_path = path;
+    t_last_path = fam;
     t_last_launches = 1;
     t_last_kernel = kernel;
     return W4A8_OK;
@@ -384,7 +457,7 @@ w4a8_status run_product_g(const int8_t *Xq, int M, int K, int ldq, const float *
                           const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
                           int ldy, cudaStream_t stream, bool after_act_pass) {
     const unsigned path = flags & W4A8_PATH_MASK;
-    if (path != W4A8_PATH_AUTO && path != W4A8_PATH_DECODE) return W4A8_ERR_UNSUPPORTED;
+    if (path != W4A8_PATH_AUTO && path_family(path) != W4A8_PATH_DECODE) return W4A8_ERR_UNSUPPORTED;
     const int tok = M <= 8 ? 8 : 16;
     const int tiles = (M + tok - 1) / tok;
     if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
@@ -418,7 +491,7 @@ w4a8_status run_product8(const int8_t *Xq, int M, int K, int ldq, const float *s
                          cudaStream_t stream, bool after_act_pass = false) {
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
-    const unsigned path = choose_path(M, K, N, flags);
+    const unsigned path = path_family(choose_path(M, K, N, flags));
     cudaError_t e = cudaSuccess;
     const char *kernel = "";
     if (path == W4A8_PATH_GENERIC) {
@@ -734,8 +807,21 @@ static w4a8_status linear_from_f32(const float *X, int M, int K, int ldx, const 
                                    const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
                                    const Workspace &ws, cudaStream_t s) {
     const unsigned path = choose_path(M, K, N, flags);
-    if (fq_eligible(M, K, N, path)) return launch_fq(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
-    const bool perm = path == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
+    const unsigned fam = path_family(path);
+    const DecodeKernel dk = fam == W4A8_PATH_DECODE ? decode_kernel_for(path, M, K, N) : DK_NONE;
+    if (fam == W4A8_PATH_DECODE && dk == DK_NONE) return W4A8_ERR_UNSUPPORTED;
+    if (dk == DK_SPLIT) {
+        // one launch: the K-split kernel quantizes its slices itself
+        cudaError_t e = launch_split(dsplit::IN_F32, nullptr, 0, nullptr, X, ldx, nullptr, 0, M, K, Wp, ldp, sw, N,
+                                     bias, flags, Y, ldy, nullptr, (flags & W4A8_STATIC_WEIGHTS) != 0, s);
+        if (e != cudaSuccess) return W4A8_ERR_CUDA;
+        t_last_path = W4A8_PATH_DECODE;
+        t_last_launches = 1;
+        t_last_kernel = "k_decode_split";
+        return W4A8_OK;
+    }
+    if (dk == DK_RING && fq_eligible(M, K, N)) return launch_fq(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, s);
+    const bool perm = fam == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
     w4a8_status st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s, perm);
     if (st != W4A8_OK) return st;
     st = run_product(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sw, N, bias, flags, Y, ldy, s, perm, true);
@@ -799,6 +885,62 @@ w4a8_status w4a8_linear_noalloc(const float *X, int M, int K, int ldx, const uin
 }
 
 size_t w4a8_noalloc_scratch_bytes(void) { return (size_t)W4A8_NOALLOC_SCRATCH_BYTES; }
+
+int w4a8_amax_parts(int N) { return N < 1 ? -1 : (N + 15) / 16; }
+
+w4a8_status w4a8_linear_chain(const float *X, int M, int K, int ldx, const float *x_amax, int x_parts,
+                              const uint8_t *Wp, int ldp, const float *sw, int N, const float *bias, unsigned flags,
+                              float *Y, int ldy, float *y_amax, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    if ((flags & W4A8_OUT_MASK) != W4A8_OUT_F32) return W4A8_ERR_INVALID_ARG;
+    w4a8_status st = check_common(M, K, N, Wp, ldp, sw, bias, flags, Y, ldy);
+    if (st != W4A8_OK) return st;
+    if (ldx < K) return W4A8_ERR_INVALID_ARG;
+    if (x_amax && (x_parts < 1 || !aligned4(x_amax))) return W4A8_ERR_INVALID_ARG;
+    if (y_amax && !aligned4(y_amax)) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) { t_last_launches = 0; t_last_kernel = ""; return W4A8_OK; }
+    if (!X || !aligned4(X)) return W4A8_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return W4A8_ERR_WORKSPACE;
+    if (workspace_bytes < w4a8_workspace_size(M, K)) return W4A8_ERR_WORKSPACE;
+    if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned path = choose_path(M, K, N, flags);
+    const unsigned fam = path_family(path);
+    const int y_parts = (N + 15) / 16;
+    if (fam == W4A8_PATH_GENERIC) {
+        dim3 grid((N + chain::GEN_THREADS - 1) / chain::GEN_THREADS, (unsigned)(M < 65535 ? M : 65535));
+        cudaError_t e = launch_pdl(chain::k_linear_generic_f32, grid, dim3(chain::GEN_THREADS), 0, s, X, M, K, ldx,
+                                   x_amax, x_parts, Wp, ldp, sw, N, bias, flags, Y, ldy, y_amax, y_parts);
+        if (e != cudaSuccess) return W4A8_ERR_CUDA;
+        t_last_path = W4A8_PATH_GENERIC;
+        t_last_launches = 1;
+        t_last_kernel = "k_linear_generic";
+        return W4A8_OK;
+    }
+    const DecodeKernel dk = fam == W4A8_PATH_DECODE ? decode_kernel_for(path, M, K, N) : DK_NONE;
+    if (fam == W4A8_PATH_DECODE && dk == DK_NONE) return W4A8_ERR_UNSUPPORTED;
+    if (dk == DK_SPLIT) {
+        cudaError_t e = launch_split(x_amax ? dsplit::IN_F32_PARTS : dsplit::IN_F32, nullptr, 0, nullptr, X, ldx,
+                                     x_amax, x_parts, M, K, Wp, ldp, sw, N, bias, flags, Y, ldy, y_amax,
+                                     (flags & W4A8_STATIC_WEIGHTS) != 0, s);
+        if (e != cudaSuccess) return W4A8_ERR_CUDA;
+        t_last_path = W4A8_PATH_DECODE;
+        t_last_launches = 1;
+        t_last_kernel = "k_decode_split";
+        return W4A8_OK;
+    }
+    // the other kernels: the activation pass and the product, then the parts
+    const Workspace ws = carve_workspace(workspace, M, K);
+    st = linear_from_f32(X, M, K, ldx, Wp, ldp, sw, N, bias, flags, Y, ldy, ws, s);
+    if (st != W4A8_OK || !y_amax) return st;
+    const unsigned launches = t_last_launches;
+    dim3 grid((y_parts + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
+    cudaError_t e = launch_pdl(chain::k_row_amax_parts, grid, dim3(128), 0, s, static_cast<const float *>(Y), M, N,
+                               ldy, y_amax, y_parts);
+    if (e != cudaSuccess) return W4A8_ERR_CUDA;
+    t_last_launches = launches + 1;
+    return W4A8_OK;
+}
 
 w4a8_status w8a8_linear(const float *X, int M, int K, int ldx, const int8_t *Wq, int ldw8,
                         const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,

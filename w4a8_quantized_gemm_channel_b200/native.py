@@ -21,11 +21,13 @@ RELU = 0x01
 OUT_F32, OUT_BF16, OUT_S32 = 0x00, 0x02, 0x04
 STATIC_WEIGHTS = 0x08
 PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TC = 0x00, 0x10, 0x20, 0x30
+PATH_DECODE_RING, PATH_DECODE_REGS, PATH_DECODE_SPLIT = 0x40, 0x50, 0x60
 MAX_K = 2097152
 
 _OUT = {"f32": OUT_F32, "bf16": OUT_BF16, "s32": OUT_S32}
 _OUT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "s32": torch.int32}
-_PATH = {"auto": PATH_AUTO, "generic": PATH_GENERIC, "decode": PATH_DECODE, "tc": PATH_TC}
+_PATH = {"auto": PATH_AUTO, "generic": PATH_GENERIC, "decode": PATH_DECODE, "tc": PATH_TC,
+         "ring": PATH_DECODE_RING, "regs": PATH_DECODE_REGS, "split": PATH_DECODE_SPLIT}
 PATH_NAMES = {v: k for k, v in _PATH.items()}
 
 class Problem(ctypes.Structure):
@@ -48,6 +50,8 @@ SIGNATURES = {
     "w4a8_linear_q": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_linear_noalloc": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P]),
     "w4a8_noalloc_scratch_bytes": (_S, []),
+    "w4a8_amax_parts": (_I, [_I]),
+    "w4a8_linear_chain": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _P, _S, _P]),
     "w8a8_ld": (_I, [_I]),
     "w8_quantize": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     "w8a8_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _U, _P, _I, _P, _S, _P]),
@@ -204,6 +208,44 @@ def w4a8_linear_q(xq: torch.Tensor, sx: torch.Tensor, k: int, wp: torch.Tensor,
                              _stream(stream)),
            "w4a8_linear_q")
     return y
+
+
+def amax_parts(n: int) -> int:
+    return lib.w4a8_amax_parts(n)
+
+
+def w4a8_linear_chain(x: torch.Tensor, wp: torch.Tensor, sw: torch.Tensor,
+                      x_amax: torch.Tensor | None = None, bias: torch.Tensor | None = None,
+                      relu: bool = False, emit_amax: bool = True, path: str = "auto",
+                      y: torch.Tensor | None = None, y_amax: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, stream=None,
+                      static_weights: bool = False):
+    """One chained Dense layer: Y[M][N] float32 as w4a8_linear, taking the
+    input's per-row abs-max parts x_amax [M][parts] (or None) and returning
+    (Y, y_amax) with y_amax [M][amax_parts(N)] (None if emit_amax is False)."""
+    ldx = _rowmajor(x, "X")
+    ldp = _rowmajor(wp, "Wp")
+    m, k = x.shape
+    n = wp.shape[0]
+    y, ldy = _out_tensor(y, m, n, "f32", x.device)
+    if emit_amax and y_amax is None:
+        y_amax = torch.empty((m, amax_parts(n)), dtype=torch.float32, device=x.device)
+    if not emit_amax:
+        y_amax = None
+    x_parts = 0
+    if x_amax is not None:
+        if x_amax.dim() != 2 or x_amax.shape[0] != m or not x_amax.is_contiguous():
+            raise ValueError("x_amax must be a contiguous [M][parts] tensor")
+        x_parts = x_amax.shape[1]
+    need = workspace_size(m, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _check(lib.w4a8_linear_chain(_ptr(x), m, k, ldx, _ptr(x_amax), x_parts, _ptr(wp), ldp, _ptr(sw), n,
+                                 _ptr(bias), flags_for(relu, "f32", path, static_weights), _ptr(y), ldy,
+                                 _ptr(y_amax), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream)),
+           "w4a8_linear_chain")
+    return y, y_amax
 
 
 def w4a8_linear_grouped(problems, relu: bool = False, out: str = "f32", stream=None,
