@@ -128,6 +128,10 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def stop(self) -> dict:
+        self.summary = self._stop()
+        return self.summary
+
+    def _stop(self) -> dict:
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -354,20 +358,30 @@ def build_graphs(torch, wl, nsteps):
     return g, full, gr
 
 
-def timed_repeats(torch, enqueue, dist=None, device=None, min_repeats=5):
+PREROLL_S = 0.3         # untimed load before a sampled region, so every clock sample is under load
+
+
+def timed_repeats(torch, enqueue, dist=None, device=None, min_repeats=5, min_s=None, clocks=None):
     """Median device time (ms) of one `enqueue()` (already warmed) over
     back-to-back repeats, each bracketed by CUDA events on the current stream;
-    repeats run until MIN_TIMED_S of device time is covered (at least
-    min_repeats, at most MAX_REPEATS; the same count on every rank). Returns
-    (median ms, repeats)."""
+    repeats run until min_s (default MIN_TIMED_S) of device time is covered
+    (at least min_repeats, at most MAX_REPEATS; the same count on every
+    rank). With `clocks`, the sampler starts before an untimed pre-roll of
+    PREROLL_S and stops right after the timed repeats. Returns (median ms,
+    repeats)."""
+    min_s = MIN_TIMED_S if min_s is None else min_s
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     enqueue()
     b.record()
     torch.cuda.synchronize()
     one = max(a.elapsed_time(b), 1e-3)
-    reps = int(min(MAX_REPEATS, max(min_repeats, -(-MIN_TIMED_S * 1e3 // one))))
+    reps = int(min(MAX_REPEATS, max(min_repeats, -(-min_s * 1e3 // one))))
     reps = int(max_over_ranks(torch, dist, float(reps), device))
+    if clocks is not None:
+        clocks.start()
+        for _ in range(int(min(MAX_REPEATS, max(1, PREROLL_S * 1e3 // one)))):
+            enqueue()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
     if dist is not None:
         dist.barrier()
@@ -377,12 +391,14 @@ def timed_repeats(torch, enqueue, dist=None, device=None, min_repeats=5):
         enqueue()
         evs[i + 1].record()
     torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.stop()
     if dist is not None:
         dist.barrier()
     return statistics.median(evs[i].elapsed_time(evs[i + 1]) for i in range(reps)), reps
 
 
-def time_steps(torch, wl, steps, warmup, dist=None, device=None):
+def time_steps(torch, wl, steps, warmup, dist=None, device=None, clocks=None):
     """Median device time (ms) of a region of exactly `steps` steps, and the
     repeat count. The timed graphs themselves run the warm-up (at least
     `warmup` steps, and every graph at least once), so no graph is replayed
@@ -397,7 +413,7 @@ def time_steps(torch, wl, steps, warmup, dist=None, device=None):
     for _ in range(max(1, -(-warmup // steps))):
         region()
     torch.cuda.synchronize()
-    return timed_repeats(torch, region, dist, device)
+    return timed_repeats(torch, region, dist, device, clocks=clocks)
 
 
 def _graph_of(torch, run):
@@ -456,7 +472,10 @@ def time_gemm_only(torch, nat, wl):
             xq, sx = xqs[i]
             lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
     g = _graph_of(torch, run)
-    ms, _ = timed_repeats(torch, g.replay, min_repeats=20)
+    # a kernel timed alone: a short burst after the device had a moment to
+    # leave the power cap the long step region may have reached
+    time.sleep(1.0)
+    ms, _ = timed_repeats(torch, g.replay, min_repeats=10, min_s=0.0)
     return ms / wl.pool
 
 
@@ -626,10 +645,8 @@ def prefill_record(args, torch, native, synth, device, props, dist, world, rank,
     Returns the record (value in TOPS, with roofline, clocks and launches)."""
     wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu, w8=w8)
     clocks = ClockSampler(device.index or 0)
-    clocks.start()
-    time.sleep(0.3)
-    ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device)
-    ck = clocks.stop()
+    ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device, clocks=clocks)
+    ck = clocks.summary
     ms = max_over_ranks(torch, dist, ms, device)
     tops = world * args.steps * wl.ops_per_step() / (ms * 1e-3) / 1e12
     g_ms = time_gemm_only(torch, native, wl)
@@ -645,7 +662,9 @@ def prefill_record(args, torch, native, synth, device, props, dist, world, rank,
            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                         "unit": "TOPS", "frac": round(achieved / peak, 4),
                         "peak_source": f"{kind} bf16_tflops (burst) x {INT8_OVER_BF16:g}, the nominal dense "
-                                       "int8/bf16 ratio (4.5 / 2.25 PFLOP/s)",
+                                       "int8/bf16 ratio (4.5 / 2.25 PFLOP/s); the kernel is timed alone, in a "
+                                       "burst of back-to-back launches",
+                        "peak_sustained": round(INT8_OVER_BF16 * float(peaks.get("bf16_tflops_sustained", 1400.0)), 1),
                         "traffic": traffic, "traffic_note": tnote,
                         "kernel": "k_gemm_tc (" + ("w8a8" if w8 else "w4a8") + "_linear_q back to back over "
                                   "rotating buffers)", "us": round(g_ms * 1e3, 2)},
@@ -679,10 +698,8 @@ def decode_record(args, torch, native, synth, device, props, dist, world, form="
     wl = DecodeWorkload(torch, native, synth, device, props.L2_cache_size, w8=form == "w8", zp=form == "zp",
                         grp=form == "grp")
     clocks = ClockSampler(device.index or 0)
-    clocks.start()
-    time.sleep(0.3)
-    ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device)
-    ck = clocks.stop()
+    ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device, clocks=clocks)
+    ck = clocks.summary
     ms = max_over_ranks(torch, dist, ms, device)
     bytes_step = wl.bytes_per_step()
     value = world * args.steps * bytes_step / (ms * 1e-3) / 1e9

@@ -26,9 +26,11 @@ NVCC_FLAGS = [
     # exactly like the method's statement.
     "-prec-div=true", "-fmad=false",
     "--expt-relaxed-constexpr",
-    # compile the kernels of the one translation unit in parallel (ptxas runs
-    # per kernel; one thread per host core)
-    "--split-compile=0",
+    # assemble the kernels of the one translation unit in parallel, one ptxas
+    # thread per host core (each kernel is still assembled on its own, so the
+    # code is the same as a serial build; nvcc's own --split-compile also
+    # splits the optimizer's module and changes the generated code)
+    "-Xptxas", "-split-compile=0",
 ]
 
 

@@ -132,10 +132,16 @@ constexpr int a_col(int slot) { return 2 * BT + slot * A_COLS; }
 // form. v = raw TMEM words, SHIFT = 4 when they hold 16*acc.
 enum { EPI_F32 = 0, EPI_BF16 = 1, EPI_S32 = 2 };
 
+// Returns true when some d = sx * sw of the chunk lies outside 2^-94..2^126,
+// where the reciprocal form is not valid (its correction needs a normal 1/d
+// and a finite f * r for |f| < 2^31); the caller then redoes the chunk with
+// the IEEE division (epi_chunk_exact), which keeps the rare path out of this
+// unrolled loop.
 template <int FMT, bool BIAS, bool RELU, int SHIFT, bool FULL>
-__device__ __forceinline__ void epi_chunk(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0, int mrem,
+__device__ __forceinline__ bool epi_chunk(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0, int mrem,
                                           int n, bool n_ok, float swn, float rswn, float bn,
                                           const float *__restrict__ tsx, const float *__restrict__ rsx) {
+    bool bad = false;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         if (!FULL && j >= mrem) break;
@@ -150,10 +156,7 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&v)[32], void *__restr
             const float q0 = __fmul_rn(f, r);
             const float e = __fmaf_rn(-q0, d, f);
             float y = __fmaf_rn(e, r, q0);
-            // The correction needs a normal 1/d and a finite f * r (|f| < 2^31):
-            // outside 2^-94 <= d <= 2^126 (extreme scales whose product is tiny,
-            // huge or overflows) take the IEEE division itself.
-            if (!(d >= 0x1p-94f && d <= 0x1p126f)) y = __fdiv_rn(f, d);
+            bad |= !(d >= 0x1p-94f && d <= 0x1p126f);
             if constexpr (BIAS) y = __fadd_rn(y, bn);
             if constexpr (RELU) y = y > 0.0f ? y : 0.0f;
             if constexpr (FMT == EPI_BF16) {
@@ -163,16 +166,41 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&v)[32], void *__restr
             }
         }
     }
+    return bad;
+}
+
+// The same chunk with y = float(acc) / (sx * sw) by IEEE division (extreme
+// scale products only).
+template <int FMT, bool BIAS, bool RELU, int SHIFT>
+__device__ __noinline__ void epi_chunk_exact(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0,
+                                             int mrem, int n, bool n_ok, float swn, float bn,
+                                             const float *__restrict__ tsx) {
+#pragma unroll 1
+    for (int j = 0; j < 32 && j < mrem; ++j) {
+        const float y0 = __fdiv_rn(__int2float_rn((int32_t)v[j] >> SHIFT), __fmul_rn(tsx[j], swn));
+        float y = y0;
+        if constexpr (BIAS) y = __fadd_rn(y, bn);
+        if constexpr (RELU) y = y > 0.0f ? y : 0.0f;
+        const size_t off = (size_t)(m0 + j) * (size_t)ldy + (size_t)n;
+        if constexpr (FMT == EPI_BF16) {
+            if (n_ok) static_cast<__nv_bfloat16 *>(Y)[off] = __float2bfloat16_rn(y);
+        } else {
+            if (n_ok) static_cast<float *>(Y)[off] = y;
+        }
+    }
 }
 
 template <int FMT, bool BIAS, bool RELU, int SHIFT>
 __device__ __forceinline__ void epi_chunk_any(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0,
                                               int mrem, int n, bool n_ok, float swn, float rswn, float bn,
                                               const float *__restrict__ tsx, const float *__restrict__ rsx) {
-    if (mrem >= 32)
-        epi_chunk<FMT, BIAS, RELU, SHIFT, true>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx);
-    else
-        epi_chunk<FMT, BIAS, RELU, SHIFT, false>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx);
+    const bool bad = mrem >= 32
+                         ? epi_chunk<FMT, BIAS, RELU, SHIFT, true>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx)
+                         : epi_chunk<FMT, BIAS, RELU, SHIFT, false>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx,
+                                                                     rsx);
+    if constexpr (FMT != EPI_S32) {
+        if (bad) epi_chunk_exact<FMT, BIAS, RELU, SHIFT>(v, Y, ldy, m0, mrem, n, n_ok, swn, bn, tsx);
+    }
 }
 
 template <int BT, int UNPACK>

@@ -273,15 +273,15 @@ w4a8_status launch_fq(const float *X, int M, int K, int ldx, const uint8_t *Wp, 
     return W4A8_OK;
 }
 
-// The cluster K-split kernel serves short layers: those whose CTAs (128
-// channels x one K slice each) fit two per SM in one wave, so that the whole
-// weight stream is requested before the dependency wait and nothing but the
-// slice's activations, the MMAs and one cluster reduction remain after it.
-// Long layers keep the persistent ring (or the register kernel), which stream
-// many waves of weights per block.
-bool split_preferred(int M, int K, int N) {
+// The cluster K-split kernel serves the chained calls (w4a8_linear_chain):
+// there it replaces the activation pass and the product with one launch.
+// Plain calls keep the persistent ring and the register kernel: measured on
+// B200 in back-to-back launches at K = N = 4096, the split kernel's exchanges
+// between the CTAs of a cluster cost more than its shorter K loop saves
+// (3.98 vs 3.26 us at M = 1, 5.77 vs 4.87 us at M = 16, INT8 input).
+bool split_preferred(int M, int K, int N, bool chained) {
     const dsplit::Plan pl = dsplit::plan(M, K, N);
-    return pl.ok && (long long)pl.nblk * pl.C <= 2LL * device_info().sm_count;
+    return chained && pl.ok && (long long)pl.nblk * pl.C <= 2LL * device_info().sm_count;
 }
 
 // On a short layer (at most two 16-channel groups per SM) whose packed rows
@@ -303,11 +303,11 @@ enum DecodeKernel { DK_NONE = 0, DK_SPLIT, DK_RING, DK_REGS };
 
 // The decode kernel for a path value of the decode family: the forced one if
 // it can run the shape (DK_NONE if not), else the rule by shape.
-DecodeKernel decode_kernel_for(unsigned path, int M, int K, int N) {
+DecodeKernel decode_kernel_for(unsigned path, int M, int K, int N, bool chained = false) {
     if (path == W4A8_PATH_DECODE_SPLIT) return dsplit::plan(M, K, N).ok ? DK_SPLIT : DK_NONE;
     if (path == W4A8_PATH_DECODE_RING) return ring_plan(M, K, N).ok ? DK_RING : DK_NONE;
     if (path == W4A8_PATH_DECODE_REGS) return DK_REGS;
-    if (split_preferred(M, K, N)) return DK_SPLIT;
+    if (split_preferred(M, K, N, chained)) return DK_SPLIT;
     if (ring_plan(M, K, N).ok && !registers_beat_ring(M, K, N)) return DK_RING;
     return DK_REGS;
 }
@@ -917,7 +917,7 @@ w4a8_status w4a8_linear_chain(const float *X, int M, int K, int ldx, const float
         t_last_kernel = "k_linear_generic";
         return W4A8_OK;
     }
-    const DecodeKernel dk = fam == W4A8_PATH_DECODE ? decode_kernel_for(path, M, K, N) : DK_NONE;
+    const DecodeKernel dk = fam == W4A8_PATH_DECODE ? decode_kernel_for(path, M, K, N, true) : DK_NONE;
     if (fam == W4A8_PATH_DECODE && dk == DK_NONE) return W4A8_ERR_UNSUPPORTED;
     if (dk == DK_SPLIT) {
         cudaError_t e = launch_split(x_amax ? dsplit::IN_F32_PARTS : dsplit::IN_F32, nullptr, 0, nullptr, X, ldx,
