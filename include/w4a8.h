@@ -328,7 +328,7 @@ W4A8_API w4a8_status w8a8_linear_q(const int8_t *Xq, int M, int K, int ldq, cons
  *   acc = sum_k xq[m][k] * (q - zp[n]),  y = float(acc) / (sx[m] * sa[n]).
  * Storage: Wp as for w4_quantize_pack ([N][ldp] bytes, two nibbles per byte,
  * even k low) holding each code as the signed nibble q - 8 (q XOR 8), pad
- * nibbles 0; the W4A8 kernels multiply those and an epilogue adds
+ * nibbles 0; the W4A8 kernels multiply those and their epilogue adds
  * -(zp - 8) * sum_k xq[m][k]. Results are defined while acc fits INT32.
  */
 
@@ -343,14 +343,14 @@ W4A8_API w4a8_status w4z_quantize_pack(const float *W, int K, int N, int ldw, ui
                               float *sa, int32_t *zp, void *stream);
 
 /* Workspace bytes of w4z_linear / w4z_linear_q for M rows, K inputs and N
- * outputs (INT8 rows, scales, row sums and the INT32 accumulators); 0 if
- * M < 0, K < 1 or N < 1. */
+ * outputs (INT8 rows, scales and row sums); 0 if M < 0, K < 1 or N < 1. */
 W4A8_API size_t w4z_workspace_size(int M, int K, int N);
 
 /*
- * w4z_linear - the zero-point layer on float32 activations: activation pass,
- * row sums, the W4A8 product on the stored codes, the zero-point epilogue
- * (four launches). Arguments, flags and errors as for w4a8_linear, with
+ * w4z_linear - the zero-point layer on float32 activations: the activation
+ * pass (which also writes the row sums), then the W4A8 product on the stored
+ * codes with the zero-point correction in its epilogue (two launches).
+ * Arguments, flags and errors as for w4a8_linear, with
  * sa/zp from w4z_quantize_pack in place of sw and a workspace of at least
  * w4z_workspace_size(M, K, N) bytes.
  */
@@ -360,7 +360,8 @@ W4A8_API w4a8_status w4z_linear(const float *X, int M, int K, int ldx,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /* w4z_linear_q - the same on INT8 activations Xq [M][ldq] with scales sx [M]
- * (three launches; the workspace holds the row sums and accumulators). */
+ * (two launches: the row sums, then the product; the workspace holds the
+ * row sums). */
 W4A8_API w4a8_status w4z_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *sx,
                          const uint8_t *Wp, int ldp, const float *sa, const int32_t *zp, int N,
                          const float *bias, unsigned flags, void *Y, int ldy,

@@ -70,8 +70,25 @@ def test_w4z_s32_bit_exact(nat, path, m, k, n):
     wp, sa, zp = oracle.w4z_quantize_pack(w)
     wpd, sad, zpd = nat.w4z_quantize_pack(dev(w))
     acc = nat.w4z_linear(dev(x), wpd, sad, zpd, out="s32", path=path)
-    assert nat.last_path() == path and nat.last_launch_count() == 4
+    # the activation pass (which writes the row sums too), then the product
+    # with the zero-point correction in its epilogue
+    assert nat.last_path() == path and nat.last_launch_count() == 2
     assert np.array_equal(host(acc), oracle.linear_z(x, wp, sa, zp, k, out="s32"))
+
+
+@pytest.mark.parametrize("path", ["split", "ring", "regs"])
+@pytest.mark.parametrize("m,k,n", [(1, 64, 16), (3, 1001, 130), (8, 4096, 64)])
+def test_w4z_every_decode_kernel(nat, path, m, k, n):
+    """The zero-point correction in the epilogue of each decode kernel: INT32
+    bit-exact and float32 within the bar, with a bias and ReLU."""
+    x, w, b = _case(m, k, n, seed=3150 + m + k)
+    w[:, 1] = np.abs(w[:, 1]) + 0.5      # a negative zero point
+    wp, sa, zp = oracle.w4z_quantize_pack(w)
+    wpd, sad, zpd = nat.w4z_quantize_pack(dev(w))
+    acc = nat.w4z_linear(dev(x), wpd, sad, zpd, out="s32", path=path)
+    assert np.array_equal(host(acc), oracle.linear_z(x, wp, sa, zp, k, out="s32"))
+    y = nat.w4z_linear(dev(x), wpd, sad, zpd, bias=dev(b), relu=True, path=path)
+    assert_f32_close(host(y), oracle.linear_z(x, wp, sa, zp, k, bias=b, relu=True), b)
 
 
 @pytest.mark.parametrize("path", PATHS)
@@ -101,7 +118,7 @@ def test_w4z_q_ignores_activation_pad_bytes(nat, path):
     xq, sx = oracle.a8_quantize_rows(x, ldq=128)
     xq[:, k:] = -77
     y = nat.w4z_linear_q(dev(xq), dev(sx), k, wpd, sad, zpd, bias=dev(b), path=path)
-    assert nat.last_launch_count() == 3
+    assert nat.last_launch_count() == 2
     assert_f32_close(host(y), oracle.linear_z(x, wp, sa, zp, k, bias=b), b)
     y2 = nat.w4z_linear(dev(x), wpd, sad, zpd, bias=dev(b), path=path)
     assert np.array_equal(host(y).view(np.uint32), host(y2).view(np.uint32))

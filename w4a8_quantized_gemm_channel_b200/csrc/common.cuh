@@ -159,4 +159,20 @@ __device__ __forceinline__ void store_out(void *__restrict__ Y, int ldy, int m, 
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return min(max(v, lo), hi); }
 
+// The zero-point form of the weights stores each code q in [0, 15] as the
+// signed nibble q - 8, so the W4A8 product gives acc' = sum_k xq (q - 8) and
+// the layer's accumulator is acc = acc' - (zp[n] - 8) * rowsum[m], rowsum[m]
+// = sum_k xq[m][k] (the "INT4" concept page, section 4.1). Product kernels
+// take these two arrays and correct in their epilogue (64-bit, then the
+// INT32 result, which the method's accumulator holds); null zp: no
+// correction (the symmetric layer).
+struct ZpArgs {
+    const int32_t *zp;
+    const int32_t *rowsum;
+};
+__device__ __forceinline__ int32_t zp_fix(int32_t acc, const ZpArgs &z, int m, int n) {
+    if (z.zp == nullptr) return acc;
+    return (int32_t)((long long)acc - ((long long)ld_dep_s32(z.zp + n) - 8) * (long long)ld_dep_s32(z.rowsum + m));
+}
+
 }  // namespace w4a8

@@ -312,7 +312,7 @@ template <bool EARLY, bool FUSED, int R, int J8>
 __global__ void __launch_bounds__(THREADS, 3)
 k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ldq, const float *sx,
               const float *X, int ldx, int vec4, int M, int K, const float *sw, int N,
-              const float *bias, unsigned flags, void *Y, int ldy, int ring_n) {
+              const float *bias, unsigned flags, void *Y, int ldy, int ring_n, ZpArgs zpa) {
     __shared__ Smem sm;
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
     const Geometry geo(K);
@@ -424,7 +424,8 @@ k_decode_ring(const __grid_constant__ CUtensorMap tm_w, const int8_t *Xq, int ld
         }
         int32_t sum;
         if (!group_reduce(sm, acc, ok, warp, g, t, abort, sum)) return;
-        if (e_ok) store_value(Y, ldy, e_tk, n0 + e_ch, sum, e_sx, e_sw, has_bias, e_b, flags);
+        if (e_ok)
+            store_value(Y, ldy, e_tk, n0 + e_ch, zp_fix(sum, zpa, e_tk, n0 + e_ch), e_sx, e_sw, has_bias, e_b, flags);
         ptx::bar_sync(1, CONSUMERS);  // red is rewritten by the next group
     }
 }

@@ -78,6 +78,7 @@ struct Params {
     float *y_amax;  // [M][y_parts] or null
     int y_parts;
     int ch;  // 128-k chunks per CTA
+    ZpArgs zpa;  // zero-point correction (null zp: none)
 };
 
 // Shared-memory row pitch of the INT8 slice: ch x 128 bytes + 16, so the
@@ -382,8 +383,8 @@ k_decode_split(const __grid_constant__ Params p) {
             for (int h = 0; h < 2; ++h) {
                 const int n = h ? nB : nA;
                 const bool ok = m_ok && (h ? okB : okA);
-                const int32_t a = tot[i][2 * h + e] >> 4;  // exact: every term is a multiple of 16
                 if (!ok) continue;
+                const int32_t a = zp_fix(tot[i][2 * h + e] >> 4, p.zpa, m, n);  // >> 4 exact: terms are multiples of 16
                 const size_t off = (size_t)m * (size_t)p.ldy + (size_t)n;
                 if (fmt == W4A8_OUT_S32) {
                     static_cast<int32_t *>(p.Y)[off] = a;

@@ -116,6 +116,7 @@ struct alignas(1024) Smem {
     uint64_t mma_done;                   // final drain of the MMA pipe
     float rsx[BT];                       // 1/sx of the epilogue's current token tile
     float tsx[BT];                       // sx of the same tokens
+    int32_t trs[BT];                     // row sums of the same tokens (zero-point form; else 0)
     uint32_t tmem_base;
     int abort;
 };
@@ -140,12 +141,15 @@ enum { EPI_F32 = 0, EPI_BF16 = 1, EPI_S32 = 2 };
 template <int FMT, bool BIAS, bool RELU, int SHIFT, bool FULL>
 __device__ __forceinline__ bool epi_chunk(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0, int mrem,
                                           int n, bool n_ok, float swn, float rswn, float bn,
-                                          const float *__restrict__ tsx, const float *__restrict__ rsx) {
+                                          const float *__restrict__ tsx, const float *__restrict__ rsx,
+                                          int32_t zpn, const int32_t *__restrict__ trs) {
     bool bad = false;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         if (!FULL && j >= mrem) break;
-        const int32_t acc = (int32_t)v[j] >> SHIFT;
+        // zero-point correction in modular INT32 arithmetic: exact whenever
+        // the corrected accumulator fits INT32, as the method's does
+        const int32_t acc = (int32_t)((uint32_t)((int32_t)v[j] >> SHIFT) - (uint32_t)zpn * (uint32_t)trs[j]);
         const size_t off = (size_t)(m0 + j) * (size_t)ldy + (size_t)n;
         if constexpr (FMT == EPI_S32) {
             if (n_ok) static_cast<int32_t *>(Y)[off] = acc;
@@ -174,10 +178,12 @@ __device__ __forceinline__ bool epi_chunk(const uint32_t (&v)[32], void *__restr
 template <int FMT, bool BIAS, bool RELU, int SHIFT>
 __device__ __noinline__ void epi_chunk_exact(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0,
                                              int mrem, int n, bool n_ok, float swn, float bn,
-                                             const float *__restrict__ tsx) {
+                                             const float *__restrict__ tsx, int32_t zpn,
+                                             const int32_t *__restrict__ trs) {
 #pragma unroll 1
     for (int j = 0; j < 32 && j < mrem; ++j) {
-        const float y0 = __fdiv_rn(__int2float_rn((int32_t)v[j] >> SHIFT), __fmul_rn(tsx[j], swn));
+        const int32_t acc = (int32_t)((uint32_t)((int32_t)v[j] >> SHIFT) - (uint32_t)zpn * (uint32_t)trs[j]);
+        const float y0 = __fdiv_rn(__int2float_rn(acc), __fmul_rn(tsx[j], swn));
         float y = y0;
         if constexpr (BIAS) y = __fadd_rn(y, bn);
         if constexpr (RELU) y = y > 0.0f ? y : 0.0f;
@@ -193,13 +199,14 @@ __device__ __noinline__ void epi_chunk_exact(const uint32_t (&v)[32], void *__re
 template <int FMT, bool BIAS, bool RELU, int SHIFT>
 __device__ __forceinline__ void epi_chunk_any(const uint32_t (&v)[32], void *__restrict__ Y, int ldy, int m0,
                                               int mrem, int n, bool n_ok, float swn, float rswn, float bn,
-                                              const float *__restrict__ tsx, const float *__restrict__ rsx) {
-    const bool bad = mrem >= 32
-                         ? epi_chunk<FMT, BIAS, RELU, SHIFT, true>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx)
-                         : epi_chunk<FMT, BIAS, RELU, SHIFT, false>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx,
-                                                                     rsx);
+                                              const float *__restrict__ tsx, const float *__restrict__ rsx,
+                                              int32_t zpn, const int32_t *__restrict__ trs) {
+    const bool bad = mrem >= 32 ? epi_chunk<FMT, BIAS, RELU, SHIFT, true>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn,
+                                                                          tsx, rsx, zpn, trs)
+                                : epi_chunk<FMT, BIAS, RELU, SHIFT, false>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn,
+                                                                           bn, tsx, rsx, zpn, trs);
     if constexpr (FMT != EPI_S32) {
-        if (bad) epi_chunk_exact<FMT, BIAS, RELU, SHIFT>(v, Y, ldy, m0, mrem, n, n_ok, swn, bn, tsx);
+        if (bad) epi_chunk_exact<FMT, BIAS, RELU, SHIFT>(v, Y, ldy, m0, mrem, n, n_ok, swn, bn, tsx, zpn, trs);
     }
 }
 
@@ -207,7 +214,7 @@ template <int BT, int UNPACK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
           int M, int N, int K, const float *__restrict__ sx, const float *__restrict__ sw,
-          const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+          const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy, ZpArgs zpa) {
     constexpr int STAGES = Cfg<BT, UNPACK>::STAGES;
     constexpr int A_SLOTS = Cfg<BT, UNPACK>::A_SLOTS;
     constexpr int W_TILE_BYTES = Cfg<BT, UNPACK>::W_TILE_BYTES;
@@ -476,6 +483,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 const float v = m < M ? ld_dep(sx + m) : 1.0f;
                 sm.tsx[c] = v;
                 sm.rsx[c] = __frcp_rn(v);
+                sm.trs[c] = (zpa.zp != nullptr && m < M) ? ld_dep_s32(zpa.rowsum + m) : 0;
             }
             // One decision for all four epilogue warps (this barrier also
             // publishes rsx): a warp that gave up must not leave the others
@@ -487,6 +495,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             const float swn = n_ok ? ld_dep(sw + n) : 1.0f;
             const float rswn = __frcp_rn(swn);
             const float bn = (bias && n_ok) ? ld_dep(bias + n) : 0.0f;
+            const int32_t zpn = (zpa.zp != nullptr && n_ok) ? ld_dep_s32(zpa.zp + n) - 8 : 0;
 #pragma unroll 1
             for (int c0 = 0; c0 < BT; c0 += 32) {
                 uint32_t v[32];
@@ -497,7 +506,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
                 constexpr int SH = Cfg<BT, UNPACK>::SHIFT;
                 const int m0 = m_base + c0;
                 const float *tsx = sm.tsx + c0, *rsx = sm.rsx + c0;
-#define W4A8_EPI(F, B, R) epi_chunk_any<F, B, R, SH>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx)
+                const int32_t *trs = sm.trs + c0;
+#define W4A8_EPI(F, B, R) epi_chunk_any<F, B, R, SH>(v, Y, ldy, m0, mrem, n, n_ok, swn, rswn, bn, tsx, rsx, zpn, trs)
                 switch (epi_mode) {
                     case 0: W4A8_EPI(EPI_F32, false, false); break;
                     case 1: W4A8_EPI(EPI_F32, false, true); break;
@@ -572,7 +582,7 @@ inline size_t smem_bytes() { return sizeof(Smem<BT, UNPACK>) + 1024; }
 template <int BT, int UNPACK>
 inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
                           const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy, int sm_count,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, ZpArgs zpa = ZpArgs{nullptr, nullptr}) {
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -598,7 +608,8 @@ inline w4a8_status launch(const int8_t *Xq, int M, int K, int ldq, const float *
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_tc<BT, UNPACK>, tm_w, tm_x, M, N, K, sx, sw, bias, flags, Y, ldy);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemm_tc<BT, UNPACK>, tm_w, tm_x, M, N, K, sx, sw, bias, flags, Y, ldy,
+                                       zpa);
     return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
 }
 
@@ -634,28 +645,30 @@ inline int pick_token_tile(int M, int N, int sm_count, bool w8 = false) {
 template <int UNPACK>
 inline w4a8_status launch_bt(int bt, const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp,
                              int ldp, const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
-                             int sm_count, cudaStream_t stream) {
-    if (bt == 64) return launch<64, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+                             int sm_count, cudaStream_t stream, ZpArgs zpa) {
+    if (bt == 64)
+        return launch<64, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream, zpa);
     if (bt == 128)
-        return launch<128, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
-    return launch<192, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream);
+        return launch<128, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream, zpa);
+    return launch<192, UNPACK>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count, stream, zpa);
 }
 }  // namespace tc
 
 inline w4a8_status launch_gemm_tc(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp,
                                   int ldp, const float *sw, int N, const float *bias, unsigned flags, void *Y,
-                                  int ldy, int sm_count, cudaStream_t stream, bool act_perm = false) {
+                                  int ldy, int sm_count, cudaStream_t stream, bool act_perm = false,
+                                  ZpArgs zpa = ZpArgs{nullptr, nullptr}) {
     const int bt = tc::pick_token_tile(M, N, sm_count);
     if (K > tc::TC_X16_MAX_K) {
         if (act_perm) return W4A8_ERR_UNSUPPORTED;
         return tc::launch_bt<tc::UNPACK_SEXT>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
-                                              stream);
+                                              stream, zpa);
     }
     if (act_perm)
         return tc::launch_bt<tc::UNPACK_X16_PERM>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
-                                                  sm_count, stream);
+                                                  sm_count, stream, zpa);
     return tc::launch_bt<tc::UNPACK_X16>(bt, Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, sm_count,
-                                         stream);
+                                         stream, zpa);
 }
 
 // W8A8 product on the tensor cores: Wq [N][ldw8] INT8 codes (ldw8 a multiple

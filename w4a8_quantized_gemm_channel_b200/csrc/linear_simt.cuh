@@ -21,7 +21,7 @@ __global__ void __launch_bounds__(128)
 k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
                  const float *__restrict__ sx,
                  const uint8_t *__restrict__ Wp, int ldp, const float *__restrict__ sw, int N,
-                 const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy) {
+                 const float *__restrict__ bias, unsigned flags, void *__restrict__ Y, int ldy, ZpArgs zpa) {
     griddep_launch_dependents();
     griddep_wait();
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
@@ -37,7 +37,7 @@ k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
             acc += ld_dep_s8(xr + k) * ((int)((b & 0xFu) ^ 8u) - 8);
             if (k + 1 < K) acc += ld_dep_s8(xr + k + 1) * ((int)((b >> 4) ^ 8u) - 8);
         }
-        store_out(Y, ldy, m, n, acc, ld_dep(sx + m), swn, bias, flags);
+        store_out(Y, ldy, m, n, zp_fix(acc, zpa, m, n), ld_dep(sx + m), swn, bias, flags);
     }
 }
 
@@ -70,10 +70,14 @@ k_linear_generic(const int8_t *__restrict__ Xq, int M, int K, int ldq,
 // brought into L2 before the wait, and loads them after it.
 // ---------------------------------------------------------------------------
 constexpr int DEC_WARPS = 8;
-// chunks per warp per batch of loads: 4 for one token group, 2 for two (the
-// activation fragments double), which keeps two blocks per SM
+// chunks per warp per batch of loads: 4, so for K <= 4096 a warp's whole
+// share of the weights is in registers from before the dependency wait, for
+// one token group and for two (the second group's activation fragments take
+// the kernel from 90 to about 120 registers, still two blocks per SM; with 2
+// chunks per batch the second batch of weight loads left HBM latency after
+// the wait)
 template <int NTG>
-constexpr int dec_unroll() { return NTG == 1 ? 4 : 2; }
+constexpr int dec_unroll() { return 4; }
 
 // Packed bytes of a row that the kernels read: codes plus pad, 16-aligned.
 __host__ __device__ __forceinline__ int packed_row_bytes(int K) { return ((K + 1) / 2 + 15) / 16 * 16; }
@@ -171,10 +175,10 @@ __device__ __forceinline__ int32_t decode_reduce(int32_t (*red)[16][8 * NTG + 1]
 // Decode kernel on INT8 activations (from the activation pass or the caller).
 // EARLY: the weights are final when the kernel starts (see above).
 template <int NTG, bool EARLY>
-__global__ void __launch_bounds__(DEC_WARPS * 32)
+__global__ void __launch_bounds__(DEC_WARPS * 32, 2)
 k_linear_decode(const int8_t *Xq, int M, int K, int ldq, const float *sx,
                 const uint8_t *Wp, int ldp, const float *sw, int N,
-                const float *bias, unsigned flags, void *Y, int ldy) {
+                const float *bias, unsigned flags, void *Y, int ldy, ZpArgs zpa) {
     constexpr int TOK = 8 * NTG;
     constexpr int UNROLL = dec_unroll<NTG>();
     static_assert(16 * TOK <= DEC_WARPS * 32, "one epilogue element per thread");
@@ -234,7 +238,7 @@ k_linear_decode(const int8_t *Xq, int M, int K, int ldq, const float *sx,
     }
 
     const int32_t s = decode_reduce<NTG>(red, acc, warp, g, t);
-    if (e_ok) store_out(Y, ldy, m0 + e_tk, n0 + e_ch, s, e_sx, e_sw, bias, flags);
+    if (e_ok) store_out(Y, ldy, m0 + e_tk, n0 + e_ch, zp_fix(s, zpa, m0 + e_tk, n0 + e_ch), e_sx, e_sw, bias, flags);
 }
 
 }  // namespace w4a8

@@ -258,13 +258,16 @@ __device__ __forceinline__ void load_unit(const float *__restrict__ x, int k, in
 }
 
 // Quantize one unit of U consecutive k (k0 = first k) and store it.
+// `sum` accumulates the unit's codes (for the zero-point form's row sums).
 template <int U, bool PERM>
-__device__ __forceinline__ void store_unit(int8_t *__restrict__ row, int k0, int K, float s, const float (&v)[U]) {
+__device__ __forceinline__ void store_unit(int8_t *__restrict__ row, int k0, int K, float s, const float (&v)[U],
+                                           int &sum) {
     if constexpr (!PERM) {
         uint32_t w = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b) w |= act_code8(v[b], s, k0 + b < K) << (8 * b);
         *reinterpret_cast<uint32_t *>(row + k0) = w;
+        sum = __dp4a((int)w, 0x01010101, sum);
     } else {
         uint32_t even = 0, odd = 0;
 #pragma unroll
@@ -273,13 +276,14 @@ __device__ __forceinline__ void store_unit(int8_t *__restrict__ row, int k0, int
             odd |= act_code8(v[2 * b + 1], s, k0 + 2 * b + 1 < K) << (8 * b);
         }
         *reinterpret_cast<uint2 *>(row + k0) = make_uint2(even, odd);
+        sum = __dp4a((int)even, 0x01010101, __dp4a((int)odd, 0x01010101, sum));
     }
 }
 
 template <int THREADS, int VPT, bool PERM>
 __global__ void __launch_bounds__(THREADS)
 k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
-            int8_t *__restrict__ Xq, int ldq, float *__restrict__ sx, int vec4) {
+            int8_t *__restrict__ Xq, int ldq, float *__restrict__ sx, int vec4, int32_t *__restrict__ rowsum) {
     constexpr int U = PERM ? 8 : 4;  // consecutive k per unit of work
     constexpr int G = VPT / U;       // units a thread keeps in registers
     static_assert(THREADS % 32 == 0 && THREADS <= 1024 && VPT % U == 0, "block shape");
@@ -320,26 +324,41 @@ k_act_quant(const float *__restrict__ X, int M, int K, int ldx,
         const float s = act_scale_from_amax(a);
         if (threadIdx.x == 0) sx[m] = s;
         int8_t *row = Xq + (size_t)m * ldq;
+        int sum = 0;
         if (in_regs) {
 #pragma unroll
             for (int i = 0; i < G; ++i) {
                 const int u = threadIdx.x + i * THREADS;
-                if (u < units) store_unit<U, PERM>(row, U * u, K, s, v[i]);
+                if (u < units) store_unit<U, PERM>(row, U * u, K, s, v[i], sum);
             }
             for (int u = threadIdx.x + G * THREADS; u < units; u += THREADS) {
                 float z[U];
 #pragma unroll
                 for (int b = 0; b < U; ++b) z[b] = 0.0f;
-                store_unit<U, PERM>(row, U * u, K, s, z);
+                store_unit<U, PERM>(row, U * u, K, s, z, sum);
             }
         } else {
             for (int u = threadIdx.x; u < units; u += THREADS) {
                 float w[U];
                 load_unit<U>(x, U * u, K, vec4 != 0, w);
-                store_unit<U, PERM>(row, U * u, K, s, w);
+                store_unit<U, PERM>(row, U * u, K, s, w, sum);
             }
         }
-        __syncthreads();  // red is reused by the next row
+        __syncthreads();  // red is reused below and by the next row
+        if (rowsum != nullptr) {
+            // sum_k xq[m][k] for the zero-point form (pad codes are 0)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) red[warp] = __int_as_float(sum);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                int t = 0;
+#pragma unroll
+                for (int i = 0; i < THREADS / 32; ++i) t += __float_as_int(red[i]);
+                rowsum[m] = t;
+            }
+            __syncthreads();
+        }
     }
 }
 

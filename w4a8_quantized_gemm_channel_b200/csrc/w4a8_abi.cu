@@ -196,7 +196,8 @@ RingPlan ring_plan(int M, int K, int N) {
 template <bool EARLY, bool FUSED, int R, int J8>
 cudaError_t launch_ring_kernel(const RingPlan &plan, const int8_t *Xq, int ldq, const float *sx, const float *X,
                                int ldx, int vec4, int M, int K, const uint8_t *Wp, int ldp, const float *sw, int N,
-                               const float *bias, unsigned flags, void *Y, int ldy, cudaStream_t s) {
+                               const float *bias, unsigned flags, void *Y, int ldy, cudaStream_t s,
+                               ZpArgs zpa = ZpArgs{nullptr, nullptr}) {
     const dbulk::Geometry geo(K);
     // the packed rows as [N][kp / 8] elements of 8 bytes, stride ldp
     CUtensorMap tm_w;
@@ -206,18 +207,18 @@ cudaError_t launch_ring_kernel(const RingPlan &plan, const int8_t *Xq, int ldq, 
     auto kern = dbulk::k_decode_ring<EARLY, FUSED, R, J8>;
     if (!raise_smem_limit(reinterpret_cast<const void *>(kern), dbulk::SMEM_BUDGET)) return cudaErrorInvalidValue;
     return launch_pdl(kern, dim3(plan.grid), dim3(dbulk::THREADS), plan.smem, s, tm_w, Xq, ldq, sx, X, ldx, vec4, M,
-                      K, sw, N, bias, flags, Y, ldy, plan.ring_n);
+                      K, sw, N, bias, flags, Y, ldy, plan.ring_n, zpa);
 }
 
 // Product on INT8 activations through the persistent decode kernel.
 cudaError_t launch_ring_q(const RingPlan &plan, bool early, const int8_t *Xq, int ldq, const float *sx, int M,
                           int K, const uint8_t *Wp, int ldp, const float *sw, int N, const float *bias,
-                          unsigned flags, void *Y, int ldy, cudaStream_t s) {
+                          unsigned flags, void *Y, int ldy, cudaStream_t s, ZpArgs zpa) {
     if (early)
         return launch_ring_kernel<true, false, 1, 1>(plan, Xq, ldq, sx, nullptr, 0, 0, M, K, Wp, ldp, sw, N,
-                                                           bias, flags, Y, ldy, s);
+                                                           bias, flags, Y, ldy, s, zpa);
     return launch_ring_kernel<false, false, 1, 1>(plan, Xq, ldq, sx, nullptr, 0, 0, M, K, Wp, ldp, sw, N, bias,
-                                                        flags, Y, ldy, s);
+                                                        flags, Y, ldy, s, zpa);
 }
 
 // Decode with the activation quantization fused in, for M <= 4: the block
@@ -318,7 +319,7 @@ DecodeKernel decode_kernel_for(unsigned path, int M, int K, int N, bool chained 
 cudaError_t launch_split(int in, const int8_t *Xq, int ldq, const float *sx, const float *X, int ldx,
                          const float *x_amax, int x_parts, int M, int K, const uint8_t *Wp, int ldp,
                          const float *sw, int N, const float *bias, unsigned flags, void *Y, int ldy,
-                         float *y_amax, bool early, cudaStream_t s) {
+                         float *y_amax, bool early, cudaStream_t s, ZpArgs zpa = ZpArgs{nullptr, nullptr}) {
     const dsplit::Plan pl = dsplit::plan(M, K, N);
     if (!pl.ok) return cudaErrorInvalidValue;
     dsplit::Params p = {};
@@ -343,6 +344,7 @@ cudaError_t launch_split(int in, const int8_t *Xq, int ldq, const float *sx, con
     p.y_amax = y_amax;
     p.y_parts = (N + 15) / 16;
     p.ch = pl.ch;
+    p.zpa = zpa;
     if (in == dsplit::IN_Q) return dsplit::launch<dsplit::IN_Q>(pl, p, early, s);
     if (in == dsplit::IN_F32) return dsplit::launch<dsplit::IN_F32>(pl, p, early, s);
     return dsplit::launch<dsplit::IN_F32_PARTS>(pl, p, early, s);
@@ -352,10 +354,12 @@ cudaError_t launch_split(int in, const int8_t *Xq, int ldq, const float *sx, con
 // after_act_pass: the launch directly follows this library's activation pass,
 // so the decode kernel may stream its weights before its dependency wait (as
 // it may when the caller passes W4A8_STATIC_WEIGHTS).
+// zpa: the zero-point correction of the product epilogues (null: none).
 w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx,
                         const uint8_t *Wp, int ldp, const float *sw, int N,
                         const float *bias, unsigned flags, void *Y, int ldy,
-                        cudaStream_t stream, bool act_perm = false, bool after_act_pass = false) {
+                        cudaStream_t stream, bool act_perm = false, bool after_act_pass = false,
+                        ZpArgs zpa = ZpArgs{nullptr, nullptr}) {
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
     const unsigned path = choose_path(M, K, N, flags);
@@ -370,14 +374,15 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
         kernel = "k_linear_generic";
         dim3 grid((N + 127) / 128, (unsigned)(M < 65535 ? M : 65535));
         e = launch_pdl(k_linear_generic, grid, dim3(128), 0, stream,
-                       Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+                       Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, zpa);
     } else if (dk == DK_SPLIT) {
         kernel = "k_decode_split";
         e = launch_split(dsplit::IN_Q, Xq, ldq, sx, nullptr, 0, nullptr, 0, M, K, Wp, ldp, sw, N, bias, flags, Y,
-                         ldy, nullptr, early, stream);
+                         ldy, nullptr, early, stream, zpa);
     } else if (dk == DK_RING) {
         kernel = "k_decode_ring";
-        e = launch_ring_q(ring_plan(M, K, N), early, Xq, ldq, sx, M, K, Wp, ldp, sw, N, bias, flags, Y, ldy, stream);
+        e = launch_ring_q(ring_plan(M, K, N), early, Xq, ldq, sx, M, K, Wp, ldp, sw, N, bias, flags, Y, ldy, stream,
+                          zpa);
     } else if (dk == DK_REGS) {
         kernel = "k_linear_decode";
         const int tok = M <= 8 ? 8 : 16;
@@ -387,12 +392,12 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
         auto kern = tok == 8 ? (early ? k_linear_decode<1, true> : k_linear_decode<1, false>)
                              : (early ? k_linear_decode<2, true> : k_linear_decode<2, false>);
         e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream,
-                       Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy);
+                       Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, zpa);
     } else if (fam == W4A8_PATH_TC) {
         kernel = "k_gemm_tc";
         if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
         w4a8_status st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
-                                        dev.sm_count, stream, act_perm);
+                                        dev.sm_count, stream, act_perm, zpa);
         if (st != W4A8_OK) return st;
     } else {
         return W4A8_ERR_INVALID_ARG;
@@ -411,15 +416,14 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
 struct ZWorkspace {
     Workspace a;
     int *rowsum;
-    int32_t *acc;
 };
 
 size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 
 size_t zworkspace_bytes(int M, int K, int N) {
+    (void)N;
     const int ldq = round_up(K, 16);
-    return round256((size_t)M * (size_t)ldq) + 2 * round256(sizeof(float) * (size_t)M) +
-           round256(sizeof(int32_t) * (size_t)M * (size_t)N) + 256;
+    return round256((size_t)M * (size_t)ldq) + 2 * round256(sizeof(float) * (size_t)M) + 256;
 }
 
 ZWorkspace carve_zworkspace(void *ws, int M, int K) {
@@ -427,28 +431,27 @@ ZWorkspace carve_zworkspace(void *ws, int M, int K) {
     z.a = carve_workspace(ws, M, K);
     uintptr_t p = reinterpret_cast<uintptr_t>(z.a.sx) + round256(sizeof(float) * (size_t)M);
     z.rowsum = reinterpret_cast<int *>(p);
-    p += round256(sizeof(int) * (size_t)M);
-    z.acc = reinterpret_cast<int32_t *>(p);
     return z;
 }
 
-// Row sums, the product on the q - 8 codes into the workspace, the
-// zero-point epilogue. after_act_pass: as for run_product.
+// The zero-point product on INT8 rows: the row sums (unless the activation
+// pass already wrote them), then the W4A8 product on the q - 8 codes with the
+// correction acc' - (zp - 8) * rowsum in its epilogue. after_act_pass: as for
+// run_product.
 w4a8_status run_product_z(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
                           const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
-                          int ldy, const ZWorkspace &zw, cudaStream_t s, bool after_act_pass) {
-    const int rows = M < 65535 ? M : 65535;
-    cudaError_t e = launch_pdl(zpt::k_row_sum8, dim3(rows), dim3(256), 0, s, Xq, M, K, ldq, zw.rowsum);
-    if (e != cudaSuccess) return W4A8_ERR_CUDA;
-    const unsigned pflags = W4A8_OUT_S32 | (flags & (W4A8_PATH_MASK | W4A8_STATIC_WEIGHTS));
-    // the row-sum kernel waits before it lets dependents start, so the
-    // product may treat the weights as final exactly as behind the activation pass
-    w4a8_status st = run_product(Xq, M, K, ldq, sx, Wp, ldp, sa, N, nullptr, pflags, zw.acc, N, s, false,
-                                 after_act_pass);
-    if (st != W4A8_OK) return st;
-    e = launch_pdl(zpt::k_zp_epilogue, dim3((N + 255) / 256, rows), dim3(256), 0, s, zw.acc, M, N, zw.rowsum, zp,
-                   sx, sa, bias, flags, Y, ldy);
-    return e == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+                          int ldy, const ZWorkspace &zw, cudaStream_t s, bool after_act_pass, bool act_perm,
+                          bool have_rowsum) {
+    if (!have_rowsum) {
+        const int rows = M < 65535 ? M : 65535;
+        cudaError_t e = launch_pdl(zpt::k_row_sum8, dim3(rows), dim3(256), 0, s, Xq, M, K, ldq, zw.rowsum);
+        if (e != cudaSuccess) return W4A8_ERR_CUDA;
+        // the row-sum kernel waits before it lets dependents start, so the
+        // product may treat the weights as final exactly as behind the activation pass
+        after_act_pass = true;
+    }
+    return run_product(Xq, M, K, ldq, sx, Wp, ldp, sa, N, bias, flags, Y, ldy, s, act_perm, after_act_pass,
+                       ZpArgs{zp, zw.rowsum});
 }
 
 // ------------------------------------------------------- group-wise INT4 ---
@@ -771,8 +774,9 @@ w4a8_status w8_quantize(const float *W, int K, int N, int ldw, int8_t *Wq, int l
     return from_cuda(cudaGetLastError());
 }
 
+// rowsum: also write sum_k xq[m][k] per row (the zero-point form), or null.
 static w4a8_status launch_act_quant(const float *X, int M, int K, int ldx, int8_t *Xq, int ldq,
-                                    float *sx, cudaStream_t s, bool perm = false) {
+                                    float *sx, cudaStream_t s, bool perm = false, int32_t *rowsum = nullptr) {
     const int vec4 = aligned16(X) && (ldx % 4 == 0);
     const int grid = M < 65535 ? M : 65535;
     cudaError_t e;
@@ -783,19 +787,24 @@ static w4a8_status launch_act_quant(const float *X, int M, int K, int ldx, int8_
     const bool wide = K > 4096 && M < 2 * device_info().sm_count;
     if (perm) {
         if (K <= 1024)
-            e = launch_pdl(k_act_quant<128, 8, true>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+            e = launch_pdl(k_act_quant<128, 8, true>, dim3(grid), dim3(128), 0, s,
+                           X, M, K, ldx, Xq, ldq, sx, vec4, rowsum);
         else if (!wide)
-            e = launch_pdl(k_act_quant<256, 16, true>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+            e = launch_pdl(k_act_quant<256, 16, true>, dim3(grid), dim3(256), 0, s,
+                           X, M, K, ldx, Xq, ldq, sx, vec4, rowsum);
         else
-            e = launch_pdl(k_act_quant<1024, 32, true>, dim3(grid), dim3(1024), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+            e = launch_pdl(k_act_quant<1024, 32, true>, dim3(grid), dim3(1024), 0, s,
+                           X, M, K, ldx, Xq, ldq, sx, vec4, rowsum);
     } else {
         if (K <= 1024)
-            e = launch_pdl(k_act_quant<128, 8, false>, dim3(grid), dim3(128), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+            e = launch_pdl(k_act_quant<128, 8, false>, dim3(grid), dim3(128), 0, s,
+                           X, M, K, ldx, Xq, ldq, sx, vec4, rowsum);
         else if (!wide)
-            e = launch_pdl(k_act_quant<256, 16, false>, dim3(grid), dim3(256), 0, s, X, M, K, ldx, Xq, ldq, sx, vec4);
+            e = launch_pdl(k_act_quant<256, 16, false>, dim3(grid), dim3(256), 0, s,
+                           X, M, K, ldx, Xq, ldq, sx, vec4, rowsum);
         else
             e = launch_pdl(k_act_quant<1024, 32, false>, dim3(grid), dim3(1024), 0, s, X, M, K, ldx, Xq, ldq, sx,
-                           vec4);
+                           vec4, rowsum);
     }
     return from_cuda(e);
 }
@@ -987,10 +996,14 @@ w4a8_status w4z_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp,
     if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
     const ZWorkspace zw = carve_zworkspace(workspace, M, K);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_act_quant(X, M, K, ldx, zw.a.xq, zw.a.ldq, zw.a.sx, s);
+    // the activation pass writes the row sums too; the tensor-core product
+    // reads its k-permuted layout
+    const bool perm = path_family(choose_path(M, K, N, flags)) == W4A8_PATH_TC && K <= tc::TC_X16_MAX_K;
+    st = launch_act_quant(X, M, K, ldx, zw.a.xq, zw.a.ldq, zw.a.sx, s, perm, zw.rowsum);
     if (st != W4A8_OK) return st;
-    st = run_product_z(zw.a.xq, M, K, zw.a.ldq, zw.a.sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, zw, s, true);
-    if (st == W4A8_OK) t_last_launches = 4;
+    st = run_product_z(zw.a.xq, M, K, zw.a.ldq, zw.a.sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, zw, s, true, perm,
+                       true);
+    if (st == W4A8_OK) t_last_launches = 2;
     return st;
 }
 
@@ -1007,8 +1020,8 @@ w4a8_status w4z_linear_q(const int8_t *Xq, int M, int K, int ldq, const float *s
     if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
     const ZWorkspace zw = carve_zworkspace(workspace, M, K);
     st = run_product_z(Xq, M, K, ldq, sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, zw,
-                       static_cast<cudaStream_t>(stream), false);
-    if (st == W4A8_OK) t_last_launches = 3;
+                       static_cast<cudaStream_t>(stream), false, false, false);
+    if (st == W4A8_OK) t_last_launches = 2;
     return st;
 }
 

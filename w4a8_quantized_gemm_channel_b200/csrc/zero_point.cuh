@@ -10,8 +10,9 @@
 // i.e. q XOR 8), pad nibbles 0, in the W4A8 packed layout. The W4A8 product
 // kernels then compute acc' = sum_k xq * (q - 8) unchanged, and
 //   acc = acc' - (zp - 8) * rowsum,  rowsum[m] = sum_k xq[m][k],
-// which the epilogue kernel here applies (in 64-bit, then dequantizes with
-// the same float32 operations as every other path).
+// which the product kernels apply in their epilogues (ZpArgs in common.cuh;
+// 64-bit, then the same float32 operations as every other path). The row sums
+// come from the activation pass, or from k_row_sum8 for INT8 input.
 #pragma once
 
 #include <climits>
@@ -156,28 +157,6 @@ k_row_sum8(const int8_t *Xq, int M, int K, int ldq, int *rowsum) {
             rowsum[m] = t;
         }
         __syncthreads();
-    }
-}
-
-// y[m][n] from acc' (the product of the q - 8 codes): acc = acc' - (zp[n] - 8)
-// * rowsum[m] in 64-bit, then the W4A8 epilogue (dequantize, bias, ReLU,
-// output format). Results are defined while acc fits INT32, as for the
-// method's INT32 accumulator. grid = (ceil(N / 256), min(M, 65535)).
-__global__ void __launch_bounds__(256)
-k_zp_epilogue(const int32_t *acc, int M, int N, const int *rowsum, const int32_t *__restrict__ zp,
-              const float *sx, const float *__restrict__ sa, const float *__restrict__ bias, unsigned flags,
-              void *Y, int ldy) {
-    griddep_wait();
-    griddep_launch_dependents();
-    const int n = blockIdx.x * 256 + threadIdx.x;
-    if (n >= N) return;
-    const bool has_bias = bias != nullptr && (flags & W4A8_OUT_MASK) != W4A8_OUT_S32;
-    const long long z8 = (long long)ld_dep_s32(zp + n) - 8;
-    const float san = ld_dep(sa + n);
-    const float b = has_bias ? ld_dep(bias + n) : 0.0f;
-    for (int m = blockIdx.y; m < M; m += gridDim.y) {
-        const long long a = (long long)ld_dep_s32(acc + (size_t)m * N + n) - z8 * (long long)ld_dep_s32(rowsum + m);
-        store_value(Y, ldy, m, n, (int32_t)a, ld_dep(sx + m), san, has_bias, b, flags);
     }
 }
 
