@@ -269,16 +269,21 @@ class PrefillWorkload:
     w4a8_linear (activation quantization + tensor-core GEMM + epilogue)."""
     name = "prefill"
 
-    def __init__(self, torch, native, synth, device, l2_bytes, relu=False, w8=False):
+    def __init__(self, torch, native, synth, device, l2_bytes, relu=False, w8=False, grp=False):
         self.torch, self.nat = torch, native
         self.w8 = w8
+        self.grp = grp  # group-wise INT4 (scale and zero point per 128 weights)
         c = synth.prefill_case()
         self.M, self.K, self.N = c.x.shape[0], c.w.shape[0], c.w.shape[1]
         self.MS = (self.M,)
         self.relu = relu
         wd = torch.from_numpy(c.w).to(device)
         self.wd = wd
-        wp, sw = native.w8_quantize(wd) if w8 else native.w4_quantize_pack(wd)
+        self.zp = None
+        if grp:
+            wp, sw, self.zp = native.w4g_quantize_pack(wd)
+        else:
+            wp, sw = native.w8_quantize(wd) if w8 else native.w4_quantize_pack(wd)
         per_set = wp.numel() + 4 * self.M * self.K + 4 * self.M * self.N
         self.pool = max(2, -(-3 * l2_bytes // per_set))
         self.wp = [wp.clone() for _ in range(self.pool)]
@@ -310,11 +315,16 @@ class PrefillWorkload:
     def step(self):
         s = self.slot
         self.slot = (self.slot + 1) % self.pool
+        if self.grp:
+            self.nat.w4g_linear(self.xs[s], self.wp[s], self.sw[s], self.zp, relu=self.relu, y=self.ys[s],
+                                workspace=self.ws[self.M])
+            return
         lin = self.nat.w8a8_linear if self.w8 else self.nat.w4a8_linear
         lin(self.xs[s], self.wp[s], self.sw[s], relu=self.relu, y=self.ys[s], workspace=self.ws[self.M])
 
     def config(self):
-        return {"workload": f"prefill single linear{' W8A8' if self.w8 else ''} M={self.M} K={self.K} "
+        form = " W8A8" if self.w8 else (" group-wise INT4 (128)" if self.grp else "")
+        return {"workload": f"prefill single linear{form} M={self.M} K={self.K} "
                             f"N={self.N}" + (" +ReLU" if self.relu else ""),
                 "M": self.M, "K": self.K, "N": self.N,
                 "l2": f"inputs larger than L2: {self.pool} distinct X/W/Y sets "
@@ -380,7 +390,7 @@ def timed_repeats(torch, enqueue, dist=None, device=None, min_repeats=5, min_s=N
     reps = int(max_over_ranks(torch, dist, float(reps), device))
     if clocks is not None:
         clocks.start()
-        for _ in range(int(min(MAX_REPEATS, max(1, PREROLL_S * 1e3 // one)))):
+        for _ in range(int(min(MAX_REPEATS, max(1, min(PREROLL_S, min_s) * 1e3 // one)))):
             enqueue()
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
     if dist is not None:
@@ -470,7 +480,10 @@ def time_gemm_only(torch, nat, wl):
     def run():
         for i in range(wl.pool):
             xq, sx = xqs[i]
-            lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
+            if wl.grp:
+                nat.w4g_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], wl.zp, relu=wl.relu, y=wl.ys[i], path="tc")
+            else:
+                lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
     g = _graph_of(torch, run)
     # a kernel timed alone: a short burst after the device had a moment to
     # leave the power cap the long step region may have reached
@@ -639,11 +652,11 @@ def run_reference(args, rank, world):
 
 
 def prefill_record(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False,
-                   cpu=None):
+                   cpu=None, grp=False):
     """Time the prefill workload: the step (w4a8_linear, activation pass
     included), the tensor-core GEMM alone, and the step through host buffers.
     Returns the record (value in TOPS, with roofline, clocks and launches)."""
-    wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu, w8=w8)
+    wl = PrefillWorkload(torch, native, synth, device, props.L2_cache_size, relu=relu, w8=w8, grp=grp)
     clocks = ClockSampler(device.index or 0)
     ms, repeats = time_steps(torch, wl, args.steps, args.warmup, dist, device, clocks=clocks)
     ck = clocks.summary
@@ -653,11 +666,14 @@ def prefill_record(args, torch, native, synth, device, props, dist, world, rank,
     peaks, kind = measured_peaks()
     peak = INT8_OVER_BF16 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
     achieved = wl.ops_per_step() / (g_ms * 1e-3) / 1e12
-    traffic, tnote = traffic_for("k_gemm_tc", "prefill" + ("-w8a8" if w8 else "") + ("-relu" if relu else ""))
+    kname = "k_gemm_tc_grp" if grp else "k_gemm_tc"
+    traffic, tnote = traffic_for(kname, "prefill" + ("-w8a8" if w8 else "") + ("-grp" if grp else "")
+                                 + ("-relu" if relu else ""))
     e2e_steps = min(args.steps, 10)
-    e_ms, h2d, d2h = time_e2e_prefill(torch, native, wl, e2e_steps) if not w8 else (None, 0, 0)
+    e_ms, h2d, d2h = time_e2e_prefill(torch, native, wl, e2e_steps) if not (w8 or grp) else (None, 0, 0)
     rec = {"value": round(tops, 2), "unit": "TOPS", "steps": args.steps, "repeats": repeats,
-           "ms_per_step": round(ms / args.steps, 6), "dtype": "s8xs8->s32" if w8 else "s8xs4->s32",
+           "ms_per_step": round(ms / args.steps, 6),
+           "dtype": "s8xs8->s32" if w8 else ("s8xu4(group zp)->f32" if grp else "s8xs4->s32"),
            "config": wl.config(),
            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                         "unit": "TOPS", "frac": round(achieved / peak, 4),
@@ -666,8 +682,8 @@ def prefill_record(args, torch, native, synth, device, props, dist, world, rank,
                                        "burst of back-to-back launches",
                         "peak_sustained": round(INT8_OVER_BF16 * float(peaks.get("bf16_tflops_sustained", 1400.0)), 1),
                         "traffic": traffic, "traffic_note": tnote,
-                        "kernel": "k_gemm_tc (" + ("w8a8" if w8 else "w4a8") + "_linear_q back to back over "
-                                  "rotating buffers)", "us": round(g_ms * 1e3, 2)},
+                        "kernel": kname + " (" + ("w8a8" if w8 else ("w4g" if grp else "w4a8"))
+                                  + "_linear_q back to back over rotating buffers)", "us": round(g_ms * 1e3, 2)},
            "gpu_launches": args.steps * wl.launches_per_step(), "clocks": ck}
     if e_ms is not None:
         rec["e2e"] = {"value": round(world * e2e_steps * wl.ops_per_step() / (e_ms * 1e-3) / 1e12, 2),
@@ -679,8 +695,10 @@ def prefill_record(args, torch, native, synth, device, props, dist, world, rank,
     return rec
 
 
-def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False, cpu=None):
-    rec = prefill_record(args, torch, native, synth, device, props, dist, world, rank, relu=relu, w8=w8, cpu=cpu)
+def run_prefill(args, torch, native, synth, device, props, dist, world, rank, relu=False, w8=False, cpu=None,
+                grp=False):
+    rec = prefill_record(args, torch, native, synth, device, props, dist, world, rank, relu=relu, w8=w8, cpu=cpu,
+                         grp=grp)
     line = {"metric": METRIC, "value": rec.pop("value"), "unit": rec.pop("unit"), "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec.pop("ms_per_step"),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rec.pop("dtype"),
@@ -957,7 +975,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=8.0,
                     help="seconds of CPU work per oracle baseline (decode, prefill sample)")
     ap.add_argument("--workload", choices=["decode", "prefill", "prefill-relu", "sweep", "gemma-stack",
-                                           "decode-w8a8", "prefill-w8a8", "decode-zp", "decode-grp"],
+                                           "decode-w8a8", "prefill-w8a8", "decode-zp", "decode-grp", "prefill-grp"],
                     default="decode",
                     help="decode (the default line: decode, with the prefill sub-record), prefill "
                          "(M=2048 K=4096 N=11008) alone, a per-shape sweep of the other workloads, the "
@@ -1014,9 +1032,10 @@ def main():
                                     f"on {threads} threads; the full-layer rate is extrapolated from that sample"}
 
     props = torch.cuda.get_device_properties(device)
-    if args.workload in ("prefill", "prefill-relu", "prefill-w8a8"):
+    if args.workload in ("prefill", "prefill-relu", "prefill-w8a8", "prefill-grp"):
         run_prefill(args, torch, native, synth, device, props, dist, world, rank,
-                    relu=args.workload == "prefill-relu", w8=args.workload == "prefill-w8a8", cpu=cpu_pf)
+                    relu=args.workload == "prefill-relu", w8=args.workload == "prefill-w8a8", cpu=cpu_pf,
+                    grp=args.workload == "prefill-grp")
         return
     if args.workload in ("decode-w8a8", "decode-zp", "decode-grp"):
         run_decode_w8a8(args, torch, native, synth, device, props, dist, world, rank,

@@ -30,9 +30,10 @@
  *    boundary and have a stride that is a multiple of 16 bytes.
  *  - Errors are returned as a w4a8_status; nothing is enqueued when an
  *    argument check fails. A CUDA launch failure returns W4A8_ERR_CUDA.
- *  - Kernels that detect an internal fault (an out-of-range index or a bounded
- *    wait that ran out) record it in a per-device status word instead of
- *    trapping; read it with w4a8_get_device_status after synchronizing.
+ *  - Kernels whose bounded wait on an asynchronous copy or tensor-core
+ *    operation runs out record W4A8_ERR_TIMEOUT in a per-device status word
+ *    instead of trapping, and return; read it with w4a8_get_device_status
+ *    after synchronizing.
  */
 #ifndef W4A8_H
 #define W4A8_H
@@ -58,8 +59,7 @@ enum {
     W4A8_ERR_UNSUPPORTED = 2,  /* no sm_100 device, or a path forced on a shape it cannot run */
     W4A8_ERR_WORKSPACE = 3,    /* workspace missing or smaller than w4a8_workspace_size() */
     W4A8_ERR_CUDA = 4,         /* a CUDA runtime call failed (e.g. a launch) */
-    W4A8_ERR_TIMEOUT = 5,      /* (device status) a bounded wait inside a kernel ran out */
-    W4A8_ERR_BOUNDS = 6        /* (device status) a kernel caught an out-of-range index */
+    W4A8_ERR_TIMEOUT = 5       /* (device status) a bounded wait inside a kernel ran out */
 };
 
 /* Flags of w4a8_linear / w4a8_linear_q. */

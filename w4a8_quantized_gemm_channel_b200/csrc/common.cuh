@@ -10,8 +10,8 @@
 namespace w4a8 {
 
 // One status word per device. Kernels record the first internal fault here
-// (bounds or a bounded wait that ran out) instead of trapping, so the context
-// stays usable and the host can read the code back. The library is one
+// (a bounded wait that ran out) instead of trapping, so the context stays
+// usable and the host can read the code back. The library is one
 // translation unit (w4a8_abi.cu includes every kernel header), so this is the
 // only definition.
 __device__ int g_device_status = 0;

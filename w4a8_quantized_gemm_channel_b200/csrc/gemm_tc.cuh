@@ -259,6 +259,31 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
     ptx::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
+    // Weight tiles of one pipeline iteration into a stage (the stage's full
+    // barrier then also waits for the activation tile).
+    auto load_weights = [&](int stage, int n_tile, int kb) {
+        ptx::mbar_arrive_expect_tx(&sm.full[stage], BT * BK + W_TILE_BYTES);
+        if constexpr (Cfg<BT, UNPACK>::W8) {
+#pragma unroll
+            for (int h = 0; h < BK / XBOX; ++h)
+                ptx::tma_load_2d(sm.wpk[stage] + h * BM * XBOX, &tm_w, kb * BK + h * XBOX, n_tile * BM,
+                                 &sm.full[stage]);
+        } else {
+            ptx::tma_load_2d(sm.wpk[stage], &tm_w, kb * (BK / 2), n_tile * BM, &sm.full[stage]);
+        }
+    };
+    // With W4A8_STATIC_WEIGHTS the weights are final at launch: the first
+    // stages' weight tiles are requested before the dependency wait (the
+    // stages are all free at the start), so they overlap the previous
+    // kernel's tail. The activations are read only after the wait.
+    const int my_iters = ((num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x) * num_kb;
+    const int pre_w = (flags & W4A8_STATIC_WEIGHTS) ? min(STAGES, my_iters) : 0;
+    if (warp == 0 && lane == 0) {
+        for (int it = 0; it < pre_w; ++it)
+            load_weights(it, ((int)blockIdx.x + (it / num_kb) * (int)gridDim.x) / tiles_m, it % num_kb);
+    }
+    __syncwarp();
+
     // Dependents may launch once every CTA of this grid is resident; the
     // activations and scales come from the previous kernel, so wait for it.
     griddep_launch_dependents();
@@ -272,18 +297,13 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUte
             uint32_t issued = 0;  // bit s: stage s has a load whose landing we have not seen
             uint32_t last_par = 0;
             bool ok = true;
+            int it = 0;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int n_tile = tile / tiles_m, m_tile = tile % tiles_m;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!ptx::mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&sm.full[stage], BT * BK + W_TILE_BYTES);
-                    if constexpr (Cfg<BT, UNPACK>::W8) {
-#pragma unroll
-                        for (int h = 0; h < BK / XBOX; ++h)
-                            ptx::tma_load_2d(sm.wpk[stage] + h * BM * XBOX, &tm_w, kb * BK + h * XBOX, n_tile * BM,
-                                             &sm.full[stage]);
-                    } else {
-                        ptx::tma_load_2d(sm.wpk[stage], &tm_w, kb * (BK / 2), n_tile * BM, &sm.full[stage]);
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    if (it >= pre_w) {
+                        if (!ptx::mbar_wait(&sm.empty[stage], phase ^ 1, abort)) { ok = false; break; }
+                        load_weights(stage, n_tile, kb);
                     }
 #pragma unroll
                     for (int h = 0; h < BK / XBOX; ++h)

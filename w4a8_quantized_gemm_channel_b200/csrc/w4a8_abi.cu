@@ -18,6 +18,7 @@
 #include "decode_split.cuh"
 #include "chain.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc_grp.cuh"
 
 namespace w4a8 {
 namespace {
@@ -456,11 +457,36 @@ w4a8_status run_product_z(const int8_t *Xq, int M, int K, int ldq, const float *
 
 // ------------------------------------------------------- group-wise INT4 ---
 // The group-wise product (any M, tiles of 8 or 16 tokens; float32 outputs).
+// The group-wise path: the tensor-core form for many rows (or W4A8_PATH_TC),
+// the decode-style kernel for few rows (or the decode family forced).
+unsigned path_g(int M, unsigned flags) {
+    const unsigned path = flags & W4A8_PATH_MASK;
+    if (path == W4A8_PATH_TC) return W4A8_PATH_TC;
+    if (path != W4A8_PATH_AUTO && path_family(path) != W4A8_PATH_DECODE) return 0;
+    if (path == W4A8_PATH_AUTO && M > 16 && tc::encode_fn() != nullptr) return W4A8_PATH_TC;
+    return W4A8_PATH_DECODE;
+}
+
+// act_perm: Xq uses the k-permuted layout (only the tensor-core form reads it).
 w4a8_status run_product_g(const int8_t *Xq, int M, int K, int ldq, const float *sx, const uint8_t *Wp, int ldp,
                           const float *sa, const int32_t *zp, int N, const float *bias, unsigned flags, void *Y,
-                          int ldy, cudaStream_t stream, bool after_act_pass) {
-    const unsigned path = flags & W4A8_PATH_MASK;
-    if (path != W4A8_PATH_AUTO && path_family(path) != W4A8_PATH_DECODE) return W4A8_ERR_UNSUPPORTED;
+                          int ldy, cudaStream_t stream, bool after_act_pass, bool act_perm = false) {
+    const unsigned path = path_g(M, flags);
+    if (path == 0) return W4A8_ERR_UNSUPPORTED;
+    if (path == W4A8_PATH_TC) {
+        if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
+        const int sms = device_info().sm_count;
+        w4a8_status st = act_perm ? tcg::launch<true>(Xq, M, K, ldq, sx, Wp, ldp, sa, zp, grp::groups_of(K), N, bias,
+                                                      flags, Y, ldy, sms, stream)
+                                  : tcg::launch<false>(Xq, M, K, ldq, sx, Wp, ldp, sa, zp, grp::groups_of(K), N, bias,
+                                                       flags, Y, ldy, sms, stream);
+        if (st != W4A8_OK) return st;
+        t_last_path = W4A8_PATH_TC;
+        t_last_launches = 1;
+        t_last_kernel = "k_gemm_tc_grp";
+        return W4A8_OK;
+    }
+    if (act_perm) return W4A8_ERR_INVALID_ARG;
     const int tok = M <= 8 ? 8 : 16;
     const int tiles = (M + tok - 1) / tok;
     if (tiles > 65535) return W4A8_ERR_UNSUPPORTED;
@@ -1048,9 +1074,11 @@ w4a8_status w4g_linear(const float *X, int M, int K, int ldx, const uint8_t *Wp,
     if (!device_info().ok) return W4A8_ERR_UNSUPPORTED;
     const Workspace ws = carve_workspace(workspace, M, K);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s);
+    // the tensor-core form reads the k-permuted INT8 layout
+    const bool perm = path_g(M, flags) == W4A8_PATH_TC;
+    st = launch_act_quant(X, M, K, ldx, ws.xq, ws.ldq, ws.sx, s, perm);
     if (st != W4A8_OK) return st;
-    st = run_product_g(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, s, true);
+    st = run_product_g(ws.xq, M, K, ws.ldq, ws.sx, Wp, ldp, sa, zp, N, bias, flags, Y, ldy, s, true, perm);
     if (st == W4A8_OK) t_last_launches = 2;
     return st;
 }
@@ -1143,7 +1171,6 @@ const char *w4a8_status_string(w4a8_status s) {
         case W4A8_ERR_WORKSPACE: return "workspace missing or too small";
         case W4A8_ERR_CUDA: return "CUDA error";
         case W4A8_ERR_TIMEOUT: return "bounded wait in a kernel ran out";
-        case W4A8_ERR_BOUNDS: return "out-of-range index caught in a kernel";
         default: return "unknown status";
     }
 }
