@@ -51,6 +51,17 @@
  * summed over the groups in increasing g in float32:
  *   y = sum_g float(sum_{k in g} xq * (q - zp[n][g])) / (sx * sa[n][g]).
  *
+ * Inputs outside the statement: non-finite values, and rows or weight
+ * columns whose scale overflows float32 (a row abs-max below 127 / FLT_MAX,
+ * a column abs-max below 7 / FLT_MAX): the pages define no scale there. Finite
+ * scales whose product sx * sw overflows or underflows stay inside it and give
+ * the IEEE quotient (acc / inf, acc / 0).
+ *
+ * Layer chaining (the minimal model's Dense -> Dense, each layer quantizing
+ * its own float32 input): a layer's input row scale comes from that row's
+ * abs-max whatever hands the maximum over, so a chain of linear() calls is
+ * the statement of a chained model (mlp() below).
+ *
  * Precision: the page's model is float32 end to end (its inputs are cast with
  * astype("float32")), and float32 decides every integer code, so each step
  * below runs in float32 with IEEE round-to-nearest. Build flags:
