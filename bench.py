@@ -473,7 +473,8 @@ def time_kernel_only(torch, nat, wl):
 
 def time_gemm_only(torch, nat, wl):
     """Device time per tensor-core GEMM launch (w4a8_linear_q on INT8
-    activations) over the rotating buffer sets (median over repeats)."""
+    activations, the kernel the library picks for the shape) over the
+    rotating buffer sets (median over repeats)."""
     xqs = [nat.a8_quantize_rows(x) for x in wl.xs]
     lin_q = nat.w8a8_linear_q if wl.w8 else nat.w4a8_linear_q
 
@@ -483,7 +484,7 @@ def time_gemm_only(torch, nat, wl):
             if wl.grp:
                 nat.w4g_linear_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], wl.zp, relu=wl.relu, y=wl.ys[i], path="tc")
             else:
-                lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i], path="tc")
+                lin_q(xq, sx, wl.K, wl.wp[i], wl.sw[i], relu=wl.relu, y=wl.ys[i])
     g = _graph_of(torch, run)
     # a kernel timed alone: a short burst after the device had a moment to
     # leave the power cap the long step region may have reached
@@ -666,7 +667,7 @@ def prefill_record(args, torch, native, synth, device, props, dist, world, rank,
     peaks, kind = measured_peaks()
     peak = INT8_OVER_BF16 * float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
     achieved = wl.ops_per_step() / (g_ms * 1e-3) / 1e12
-    kname = "k_gemm_tc_grp" if grp else "k_gemm_tc"
+    kname = native.last_kernel()  # the product kernel the library picked for this shape
     traffic, tnote = traffic_for(kname, "prefill" + ("-w8a8" if w8 else "") + ("-grp" if grp else "")
                                  + ("-relu" if relu else ""))
     e2e_steps = min(args.steps, 10)
@@ -830,7 +831,7 @@ def run_sweep(torch, native, synth, device, props):
         frac = max(gbs / hbm, tops / tc)
         print(json.dumps({"shape": name, "M": m, "K": k, "N": n, "us": round(us, 3),
                           "GBs": round(gbs, 1), "TOPS": round(tops, 2), "roofline_frac": round(frac, 4),
-                          "path": native.last_path()}), flush=True)
+                          "path": native.last_path(), "kernel": native.last_kernel()}), flush=True)
         del wps, sws, wp, sw, x, y, ws, g
         torch.cuda.empty_cache()
 

@@ -79,12 +79,19 @@ enum {
 #define W4A8_PATH_AUTO     0x00u
 #define W4A8_PATH_GENERIC  0x10u /* CUDA-core kernel, any shape */
 #define W4A8_PATH_DECODE   0x20u /* weight-streaming kernel for few rows (M <= 16 per tile), picked by shape */
-#define W4A8_PATH_TC       0x30u /* tcgen05 tensor-core GEMM (INT32 accumulators in TMEM) */
+#define W4A8_PATH_TC       0x30u /* tcgen05 tensor-core GEMM (INT32 accumulators in TMEM); forced: the one-SM
+                                    * k_gemm_tc. AUTO picks the CTA-pair k_gemm_tc_pair for INT4 layers of
+                                    * M >= 1024, N >= 512, K <= 131072 and k_gemm_tc otherwise. */
 /* One kernel of the decode family, forced (W4A8_ERR_UNSUPPORTED where it
  * cannot run the shape); w4a8_last_path reports them as W4A8_PATH_DECODE. */
 #define W4A8_PATH_DECODE_RING  0x40u /* k_decode_ring: persistent TMA ring, M <= 8, K <= 131072 */
 #define W4A8_PATH_DECODE_REGS  0x50u /* k_linear_decode: weights in registers, any M in tiles of 16 */
 #define W4A8_PATH_DECODE_SPLIT 0x60u /* k_decode_split: cluster K-split, M <= 16, K <= 8192 */
+/* Forced two-SM tensor-core GEMM (k_gemm_tc_pair: tcgen05.mma cta_group::2 on
+ * a CTA pair, 256 channels x 192 tokens per tile), INT4 layers with
+ * K <= 131072 only (else W4A8_ERR_UNSUPPORTED); w4a8_last_path reports it as
+ * W4A8_PATH_TC. */
+#define W4A8_PATH_TC_PAIR  0x70u
 #define W4A8_PATH_MASK     0x70u
 
 /* Largest K whose INT32 accumulator cannot overflow: 127 * 8 * K < 2^31. */

@@ -19,6 +19,7 @@
 #include "chain.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_grp.cuh"
+#include "gemm_tc_pair.cuh"
 
 namespace w4a8 {
 namespace {
@@ -114,13 +115,15 @@ w4a8_status check_common(int M, int K, int N, const uint8_t *Wp, int ldp, const 
     const size_t esz = fmt == W4A8_OUT_BF16 ? 2 : 4;
     if ((reinterpret_cast<uintptr_t>(Y) & (esz - 1)) != 0) return W4A8_ERR_INVALID_ARG;
     if (flags & ~(W4A8_RELU | W4A8_OUT_MASK | W4A8_STATIC_WEIGHTS | W4A8_PATH_MASK)) return W4A8_ERR_INVALID_ARG;
-    if ((flags & W4A8_PATH_MASK) > W4A8_PATH_DECODE_SPLIT) return W4A8_ERR_INVALID_ARG;
     return W4A8_OK;
 }
 
 // The family (generic, decode, tensor core) of a path value: the forced
 // decode kernels belong to the decode family.
-inline unsigned path_family(unsigned path) { return path >= W4A8_PATH_DECODE_RING ? W4A8_PATH_DECODE : path; }
+inline unsigned path_family(unsigned path) {
+    if (path == W4A8_PATH_TC_PAIR) return W4A8_PATH_TC;
+    return path >= W4A8_PATH_DECODE_RING ? W4A8_PATH_DECODE : path;
+}
 
 // Kernel selection by shape. Few rows: the layer is a weight stream, so the
 // decode kernel; many rows: the tensor-core GEMM; tiny problems: generic.
@@ -132,6 +135,16 @@ unsigned choose_path(int M, int K, int N, unsigned flags) {
     if (M <= 16) return W4A8_PATH_DECODE;
     if (tc_supported(M, K, N)) return W4A8_PATH_TC;
     return W4A8_PATH_DECODE;
+}
+
+// The tensor-core product on a CTA pair (k_gemm_tc_pair) rather than on one
+// SM (k_gemm_tc): measured on B200 it is faster from M = 2048 rows up
+// (1987 against 1893 TOPS at M = 2048, K = 4096, N = 11008; 2050 against
+// 1805 at K = 11008, N = 4096; 2030 against 1970 at M = 8192) and slower at
+// M = 512 (1147 against 1259), where its 160-token tiles leave the last round
+// of the grid mostly idle.
+bool pair_preferred(int M, int K, int N) {
+    return M >= 1024 && N >= 512 && K <= tc::TC_X16_MAX_K;
 }
 
 // Kernels that take more than the default 48 KB of shared memory need the
@@ -395,10 +408,21 @@ w4a8_status run_product(const int8_t *Xq, int M, int K, int ldq, const float *sx
         e = launch_pdl(kern, grid, dim3(DEC_WARPS * 32), 0, stream,
                        Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, zpa);
     } else if (fam == W4A8_PATH_TC) {
-        kernel = "k_gemm_tc";
         if (!tc_supported(M, K, N)) return W4A8_ERR_UNSUPPORTED;
-        w4a8_status st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
-                                        dev.sm_count, stream, act_perm, zpa);
+        w4a8_status st;
+        const bool forced = (flags & W4A8_PATH_MASK) != 0;
+        if (path == W4A8_PATH_TC_PAIR || (!forced && pair_preferred(M, K, N))) {
+            kernel = "k_gemm_tc_pair";
+            if (K > tc::TC_X16_MAX_K) return W4A8_ERR_UNSUPPORTED;
+            st = act_perm ? tcp::launch<tc::UNPACK_X16_PERM>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+                                                             dev.sm_count, stream, zpa)
+                          : tcp::launch<tc::UNPACK_X16>(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy,
+                                                        dev.sm_count, stream, zpa);
+        } else {
+            kernel = "k_gemm_tc";
+            st = launch_gemm_tc(Xq, M, K, ldq, sx, Wp, ldp, sw, N, bias, flags, Y, ldy, dev.sm_count, stream,
+                                act_perm, zpa);
+        }
         if (st != W4A8_OK) return st;
     } else {
         return W4A8_ERR_INVALID_ARG;
@@ -520,6 +544,7 @@ w4a8_status run_product8(const int8_t *Xq, int M, int K, int ldq, const float *s
                          cudaStream_t stream, bool after_act_pass = false) {
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
+    if ((flags & W4A8_PATH_MASK) == W4A8_PATH_TC_PAIR) return W4A8_ERR_UNSUPPORTED;  // INT4 codes only
     const unsigned path = path_family(choose_path(M, K, N, flags));
     cudaError_t e = cudaSuccess;
     const char *kernel = "";

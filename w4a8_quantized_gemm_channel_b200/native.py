@@ -22,12 +22,14 @@ OUT_F32, OUT_BF16, OUT_S32 = 0x00, 0x02, 0x04
 STATIC_WEIGHTS = 0x08
 PATH_AUTO, PATH_GENERIC, PATH_DECODE, PATH_TC = 0x00, 0x10, 0x20, 0x30
 PATH_DECODE_RING, PATH_DECODE_REGS, PATH_DECODE_SPLIT = 0x40, 0x50, 0x60
+PATH_TC_PAIR = 0x70
 MAX_K = 2097152
 
 _OUT = {"f32": OUT_F32, "bf16": OUT_BF16, "s32": OUT_S32}
 _OUT_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "s32": torch.int32}
 _PATH = {"auto": PATH_AUTO, "generic": PATH_GENERIC, "decode": PATH_DECODE, "tc": PATH_TC,
-         "ring": PATH_DECODE_RING, "regs": PATH_DECODE_REGS, "split": PATH_DECODE_SPLIT}
+         "ring": PATH_DECODE_RING, "regs": PATH_DECODE_REGS, "split": PATH_DECODE_SPLIT,
+         "tc2": PATH_TC_PAIR}
 PATH_NAMES = {v: k for k, v in _PATH.items()}
 
 class Problem(ctypes.Structure):
