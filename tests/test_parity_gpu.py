@@ -68,6 +68,21 @@ def test_quantize_pack_bit_exact(nat, k, n):
     assert np.array_equal(host(wp), wp_ref)
 
 
+@pytest.mark.parametrize("k,n", [(1, 32), (257, 40), (600, 64), (4097, 96), (6912, 64), (12288, 32),
+                                 (12289, 32), (8192, 36)])
+def test_quantize_pack_panel_path_bit_exact(nat, k, n):
+    """Shapes around the single-pass (cluster panel) form's limits: one slice,
+    a partial 32-channel panel, a cluster whose last slice lies past K, the
+    largest K it takes (12288) and the first it hands to the two-pass form."""
+    w = synth.linear_weights(k, n, 0.02, seed=150 + k + n)
+    w[:, 3] = 0.0                          # an all-zero output channel
+    w[k // 2, 5] = 0.5                     # a column's maximum in the middle slice
+    wp, sw = nat.w4_quantize_pack(dev(w))
+    wp_ref, sw_ref = oracle.w4_quantize_pack(w)
+    assert np.array_equal(host(sw).view(np.uint32), sw_ref.view(np.uint32))
+    assert np.array_equal(host(wp), wp_ref)
+
+
 def test_quantize_pack_wide_stride_and_padding(nat):
     k, n = 77, 20
     w = synth.linear_weights(k, 24, 0.02, seed=7)     # ldw = 24 > N
@@ -77,6 +92,16 @@ def test_quantize_pack_wide_stride_and_padding(nat):
     nat.w4_quantize_pack(wd, wp=wp)
     wp_ref, _ = oracle.w4_quantize_pack(np.ascontiguousarray(w[:, :n]), ldp=ldp)
     assert np.array_equal(host(wp), wp_ref)          # pad bytes overwritten with 0
+    # a row stride much wider than the codes need, on a 16-byte aligned
+    # layout (single-pass form): the bytes past the cluster's rows are zeroed
+    k, n = 600, 40
+    w = synth.linear_weights(k, 48, 0.02, seed=8)
+    wd = dev(w)[:, :n]
+    ldp = 1024
+    wp = torch.full((n, ldp), 0xAB, dtype=torch.uint8, device="cuda")
+    nat.w4_quantize_pack(wd, wp=wp)
+    wp_ref, _ = oracle.w4_quantize_pack(np.ascontiguousarray(w[:, :n]), ldp=ldp)
+    assert np.array_equal(host(wp), wp_ref)
 
 
 # -------------------------------------------------------- activations ---

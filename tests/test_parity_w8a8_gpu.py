@@ -47,6 +47,20 @@ def test_w8_quantize_bit_exact(nat, k, n):
     assert np.array_equal(host(swd).view(np.uint32), sw.view(np.uint32))
 
 
+@pytest.mark.parametrize("k,n", [(1, 32), (257, 40), (4097, 96), (12288, 32), (12289, 32)])
+def test_w8_quantize_panel_path_bit_exact(nat, k, n):
+    """Shapes around the single-pass (cluster panel) form's limits, as for the
+    INT4 weights: a partial panel, a last slice past K, K = 12288 and the first
+    K handed to the two-pass form."""
+    w = synth.linear_weights(k, n, 0.02, seed=2050 + k + n)
+    w[:, 3] = 0.0
+    w[k // 2, 5] = 0.5
+    q8, sw = oracle.w8_quantize(w)
+    wqd, swd = nat.w8_quantize(dev(w))
+    assert np.array_equal(host(wqd), q8)
+    assert np.array_equal(host(swd).view(np.uint32), sw.view(np.uint32))
+
+
 def test_w8_quantize_wide_stride_writes_zero_pad(nat):
     """Rows wider than round_up(K, 16): every byte from K on is written 0."""
     k, n = 37, 20
@@ -54,6 +68,13 @@ def test_w8_quantize_wide_stride_writes_zero_pad(nat):
     wq = torch.full((n, 96), 77, dtype=torch.int8, device="cuda")
     nat.w8_quantize(dev(w), wq=wq)
     q8, _ = oracle.w8_quantize(w, ldw8=96)
+    assert np.array_equal(host(wq), q8)
+    # aligned layout (single-pass form) with a row stride past the cluster's rows
+    k, n = 300, 32
+    w = synth.linear_weights(k, n, 0.02, seed=2011)
+    wq = torch.full((n, 1024), 77, dtype=torch.int8, device="cuda")
+    nat.w8_quantize(dev(w), wq=wq)
+    q8, _ = oracle.w8_quantize(w, ldw8=1024)
     assert np.array_equal(host(wq), q8)
 
 

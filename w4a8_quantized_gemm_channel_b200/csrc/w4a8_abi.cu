@@ -20,6 +20,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_tc_grp.cuh"
 #include "gemm_tc_pair.cuh"
+#include "quant_pack_panel.cuh"
 
 namespace w4a8 {
 namespace {
@@ -707,6 +708,9 @@ w4a8_status w4_quantize_pack(const float *W, int K, int N, int ldw, uint8_t *Wp,
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // One pass over W (cluster panels in shared memory) where TMA can tile
+    // the layout and a slice fits; the two-pass form otherwise.
+    if (qpp::eligible(W, K, ldw)) return qpp::launch<4>(W, K, N, ldw, Wp, ldp, sw, s);
     unsigned *amax = reinterpret_cast<unsigned *>(sw);
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * (size_t)N, s);
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
@@ -797,6 +801,9 @@ w4a8_status w8_quantize(const float *W, int K, int N, int ldw, int8_t *Wq, int l
     const DeviceInfo &dev = device_info();
     if (!dev.ok) return W4A8_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // one pass over W where the layout allows it, as for the INT4 weights
+    if (qpp::eligible(W, K, ldw))
+        return qpp::launch<8>(W, K, N, ldw, reinterpret_cast<uint8_t *>(Wq), ldw8, sw, s);
     unsigned *amax = reinterpret_cast<unsigned *>(sw);
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float) * (size_t)N, s);
     if (e != cudaSuccess) return W4A8_ERR_CUDA;
