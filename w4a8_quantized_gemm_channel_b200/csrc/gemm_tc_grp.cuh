@@ -15,7 +15,7 @@
 //    group is one 128-k activation box: 4 MMAs) and alternates between two
 //    accumulator buffers, committing each group to the epilogue;
 //  * the epilogue drains every group: z += float(acc_g) * (1 / sa[n][g]) in
-//    float32 registers (acc_g is at most 128 * 127 * 15 in size, exact in
+//    float32 registers, each warp on its own barrier wait (acc_g is at most 128 * 127 * 15 in size, exact in
 //    float32), and at the end of the tile y = z * (1 / sx[m]), bias, ReLU.
 // Factoring 1 / sx out of the group sum leaves one conversion and one FMA
 // per output and group. The float32 result differs from a sequential sum of
@@ -211,20 +211,27 @@ k_gemm_tc_grp(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         const int r = q * 32 + lane;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         bool ok = true;
+        // the two groups' zero points of an iteration, fetched one iteration
+        // of this warpgroup ahead so their latency hides behind the unpack
+        auto zero_points = [&](int it, int32_t (&z)[2]) {
+            const int kb = it % num_kb;
+            const int tile = (int)blockIdx.x + (it / num_kb) * (int)gridDim.x;
+            const int n = (tile / tiles_m) * BM + r;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int gi = 2 * kb + h;
+                z[h] = (it < total && n < N && gi < ng) ? ld_dep_s32(zp + (size_t)n * ng + gi) - 8 : 0;
+            }
+        };
+        int32_t z8_next[2];
+        zero_points(wg, z8_next);
         for (int it = wg; it < total && ok; it += UNPACK_WG) {
             const int stage = it % STAGES;
             const uint32_t phase = (uint32_t)(it / STAGES) & 1u;
             const int slot = it % A_SLOTS;
             const int kb = it % num_kb;
-            const int tile = (int)blockIdx.x + (it / num_kb) * (int)gridDim.x;
-            const int n = (tile / tiles_m) * BM + r;
-            // the two groups' zero points (fetched while the stage lands)
-            int32_t z8[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int gi = 2 * kb + h;
-                z8[h] = (n < N && gi < ng) ? ld_dep_s32(zp + (size_t)n * ng + gi) - 8 : 0;
-            }
+            const int32_t z8[2] = {z8_next[0], z8_next[1]};
+            zero_points(it + UNPACK_WG, z8_next);
             bool got = ptx::mbar_wait(&sm.full[stage], phase, abort);
             if (got && it >= A_SLOTS) {
                 const int j = it - A_SLOTS;
@@ -298,20 +305,27 @@ k_gemm_tc_grp(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
                 const int m = m_base + c;
                 sm.rsx[c] = __frcp_rn(m < M ? ld_dep(sx + m) : 1.0f);
             }
+            // publishes rsx (the previous tile's readers are past the barrier
+            // at its end)
+            ptx::bar_sync(1, EPI_THREADS);
             const int n = n_tile * BM + q * 32 + lane;
             const bool n_ok = n < N;
             float z[TOK_PER_THREAD];
 #pragma unroll
             for (int j = 0; j < TOK_PER_THREAD; ++j) z[j] = 0.0f;
             float rsa = n_ok ? __frcp_rn(ld_dep(sa + (size_t)n * ng)) : 0.0f;
+            // Each warp drains its share of every group on its own (a
+            // barrier of all eight warps per group cost more than the drain);
+            // the warps agree on the outcome once per tile, below.
             for (int g = 0; g < ng; ++g) {
                 const float rsa_next = (n_ok && g + 1 < ng) ? __frcp_rn(ld_dep(sa + (size_t)n * ng + g + 1)) : 0.0f;
-                // one decision for all epilogue warps (also publishes rsx)
-                if (!ptx::bar_and(1, EPI_THREADS, ptx::mbar_wait(&sm.acc_full[gbuf], gphase, abort))) {
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&sm.acc_full[gbuf], gphase, abort))) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
+                // 16 columns per TMEM load (z and one load fit the 96 registers
+                // a thread of this 640-thread block gets)
 #pragma unroll
                 for (int c = 0; c < TOK_PER_THREAD / 16; ++c) {
                     uint32_t v[16];
@@ -328,7 +342,9 @@ k_gemm_tc_grp(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
                 if (++gbuf == 2) { gbuf = 0; gphase ^= 1u; }
                 rsa = rsa_next;
             }
-            if (!ok) break;
+            // one decision for all epilogue warps: a warp that gave up must not
+            // leave the others waiting at the named barriers
+            if (!ptx::bar_and(1, EPI_THREADS, ok)) break;
             const float bn = (bias != nullptr && n_ok) ? ld_dep(bias + n) : 0.0f;
 #pragma unroll
             for (int j = 0; j < TOK_PER_THREAD; ++j) {
