@@ -32,6 +32,44 @@ def test_library_exports_every_declared_symbol():
         assert name in native.SIGNATURES, name
 
 
+def header_defines():
+    """#define NAME value (integer literals) and the status enum of the header."""
+    text = open(HEADER).read()
+    out = {}
+    pat = r"^#define\s+(W[48]A8_\w+)\s+\(?\s*(0x[0-9a-fA-F]+|\d+)u?(?:\s*<<\s*(\d+))?"
+    for name, val, shift in re.findall(pat, text, re.M):
+        out[name] = int(val, 0) << (int(shift) if shift else 0)
+    for name, val in re.findall(r"^\s+(W4A8_(?:OK|ERR_\w+))\s*=\s*(\d+)", text, re.M):
+        out[name] = int(val)
+    return out
+
+
+def test_binding_constants_match_the_header():
+    """The binding's flag, path and status values and size limits are the
+    header's (a drift would make the Python side ask for another kernel)."""
+    from w4a8_quantized_gemm_channel_b200 import native
+    d = header_defines()
+    pairs = {"RELU": "W4A8_RELU", "OUT_F32": "W4A8_OUT_F32", "OUT_BF16": "W4A8_OUT_BF16",
+             "OUT_S32": "W4A8_OUT_S32", "STATIC_WEIGHTS": "W4A8_STATIC_WEIGHTS",
+             "PATH_AUTO": "W4A8_PATH_AUTO", "PATH_GENERIC": "W4A8_PATH_GENERIC",
+             "PATH_DECODE": "W4A8_PATH_DECODE", "PATH_TC": "W4A8_PATH_TC",
+             "PATH_DECODE_RING": "W4A8_PATH_DECODE_RING", "PATH_DECODE_REGS": "W4A8_PATH_DECODE_REGS",
+             "PATH_DECODE_SPLIT": "W4A8_PATH_DECODE_SPLIT", "PATH_TC_PAIR": "W4A8_PATH_TC_PAIR",
+             "MAX_K": "W4A8_MAX_K", "OK": "W4A8_OK", "ERR_INVALID_ARG": "W4A8_ERR_INVALID_ARG",
+             "ERR_UNSUPPORTED": "W4A8_ERR_UNSUPPORTED", "ERR_WORKSPACE": "W4A8_ERR_WORKSPACE",
+             "ERR_CUDA": "W4A8_ERR_CUDA", "ERR_TIMEOUT": "W4A8_ERR_TIMEOUT"}
+    for py, c in pairs.items():
+        assert c in d, c
+        assert getattr(native, py) == d[c], (py, getattr(native, py), d[c])
+    # the no-allocation scratch size, as the library reports it
+    assert native.NOALLOC_SCRATCH_BYTES == d["W4A8_NOALLOC_SCRATCH_BYTES"]
+    assert native.lib.w4a8_noalloc_scratch_bytes() == d["W4A8_NOALLOC_SCRATCH_BYTES"]
+    # every forced path value fits the path mask
+    for name in pairs.values():
+        if name.startswith("W4A8_PATH_"):
+            assert d[name] & ~d["W4A8_PATH_MASK"] == 0
+
+
 def test_size_queries():
     from w4a8_quantized_gemm_channel_b200 import native
     import oracle
