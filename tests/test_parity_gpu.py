@@ -311,6 +311,27 @@ def test_gemma_stack_shapes_sampled(nat):
             _sampled_check(nat, x, w, wpd, swd, rows, cols)
 
 
+@pytest.mark.parametrize("path", ["tc", "auto"])
+def test_prefill_full_size_int32_and_bf16_sampled(nat, path):
+    """M = 2048, K = 4096, N = 11008 with INT32 and bf16 outputs, through the
+    one-SM kernel (forced "tc") and the kernel the library picks (the CTA
+    pair at this shape): sampled rows x channels against the oracle, INT32
+    bit-exact and bf16 within 1 ulp."""
+    c = synth.prefill_case()
+    wpd, swd = nat.w4_quantize_pack(dev(c.w))
+    rng = synth.rng_for(12, 12)
+    rows = np.unique(np.concatenate([[0, 1, 2047], rng.integers(0, 2048, size=8)]))
+    cols = np.unique(np.concatenate([[0, 255, 256, 11007], rng.integers(0, 11008, size=60)]))
+    wp_s = host(wpd)[cols]
+    sw_s = host(swd)[cols]
+    acc = host(nat.w4a8_linear(dev(c.x), wpd, swd, out="s32", path=path))
+    assert nat.last_kernel() == ("k_gemm_tc" if path == "tc" else "k_gemm_tc_pair")
+    assert np.array_equal(acc[np.ix_(rows, cols)], oracle.linear(c.x[rows], wp_s, sw_s, c.x.shape[1], out="s32"))
+    yb = host(nat.w4a8_linear(dev(c.x), wpd, swd, out="bf16", relu=True, path=path).view(torch.int16))
+    ref = oracle.linear(c.x[rows], wp_s, sw_s, c.x.shape[1], relu=True, out="bf16")
+    assert_bf16_within_ulp(yb[np.ix_(rows, cols)], ref)
+
+
 def test_prefill_full_size_sampled(nat):
     """Prefill single linear at full size (M=2048, K=4096, N=11008), plain and
     with the fused ReLU; sampled rows x channels recomputed by the oracle."""
@@ -529,8 +550,13 @@ def test_grouped_decode_matches_single_calls(nat, out):
         a = host(y.view(torch.int32) if out != "bf16" else y.view(torch.int16))
         b1 = host(y1.view(torch.int32) if out != "bf16" else y1.view(torch.int16))
         assert np.array_equal(a, b1)
+        k = x.shape[1]
         if out == "s32":
-            assert np.array_equal(host(y), oracle.linear(x, wp, sw, x.shape[1], out="s32"))
+            assert np.array_equal(host(y), oracle.linear(x, wp, sw, k, out="s32"))
+        elif out == "bf16":
+            assert_bf16_within_ulp(a, oracle.linear(x, wp, sw, k, bias=b, relu=relu, out="bf16"))
+        else:
+            assert_f32_close(host(y), oracle.linear(x, wp, sw, k, bias=b, relu=relu), b)
 
 
 def test_grouped_decode_many_problems_and_static_weights(nat):
