@@ -254,3 +254,18 @@ def test_group_wise_calls_check_arguments_before_the_device():
     assert call(zp=None) == 1 and call(ldp=144) == 1 and call(ws=None) == 3
     assert call(M=0) == 0
     assert lib.w4g_quantize_pack(16, k, n, n, 4096, 160, 64, None, None) == 1
+
+
+def test_no_multicast_bulk_loads_in_the_kernels():
+    """No TMA or bulk copy in the kernel sources multicasts across a cluster:
+    every load lands in the issuing CTA's own shared memory (the CTA-pair
+    GEMM multicasts only its tcgen05.commit mbarrier arrives)."""
+    csrc = os.path.join(ROOT, "w4a8_quantized_gemm_channel_b200", "csrc")
+    bad = []
+    for name in sorted(os.listdir(csrc)):
+        if not name.endswith((".cu", ".cuh")):
+            continue
+        for i, line in enumerate(open(os.path.join(csrc, name)), 1):
+            if "cp.async.bulk" in line and "multicast" in line:
+                bad.append(f"{name}:{i}")
+    assert not bad, bad
